@@ -1,0 +1,493 @@
+"""Benchmark: effective prefill TFLOP/s (and speedup over the same kernel with
+every window open, alpha = inf) on one Qwen2.5-7B-shaped attention layer
+(batch 1, 28 query / 4 kv heads, d = 128, 8192 tokens, bf16, theta = 1e7,
+alpha = 1), plus decode GB/s at a 1,048,576-token cache.
+
+One step = the whole prefill hot path on one input: RoPE of q and k (fp64
+angles), windowed QK on the tensor cores, online softmax, P.V, epilogue and the
+skipped-pair counter.  Effective FLOPs count only the query-key pairs inside
+their window (4 FLOP per active pair) plus P.V (2d FLOP per causal element);
+the exponentials are not counted.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own independent layer (weak scaling; no
+collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from rope_frequency_sparse_b200 import atf, synth  # noqa: E402
+
+HEADLINE = "layer_8k"
+METRIC = "effective prefill TFLOP/s (alpha=1; active query-key pairs + P.V counted)"
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ accounting (host integers)
+
+def window_table(d, theta, alpha):
+    return [int(w) for w in atf.atf_windows(d, theta, alpha)]
+
+
+def prefill_flops(w: synth.Workload, alpha: float, seq: int | None = None) -> tuple[int, int, int]:
+    """(effective FLOPs, dense FLOPs, skipped pairs) of a causal prefill over `seq` tokens."""
+    S = w.seq if seq is None else seq
+    P = S * (S + 1) // 2
+    W = window_table(w.d, w.theta, alpha)
+    skipped = sum((S - 1 - x) * (S - x) // 2 for x in W if x < S - 1)
+    active = (w.d // 2) * P - skipped
+    eff = w.batch * w.q_heads * (4 * active + 2 * w.d * P)
+    dense = w.batch * w.q_heads * (4 * (w.d // 2) * P + 2 * w.d * P)
+    return eff, dense, w.q_heads * skipped * w.batch
+
+
+def row_flops(w: synth.Workload, alpha: float, m: int) -> int:
+    W = window_table(w.d, w.theta, alpha)
+    active = sum(min(m, x) + 1 for x in W)  # pairs i with (m - n) <= W_i over n = 0..m
+    return 4 * active + 2 * w.d * (m + 1)
+
+
+def decode_bytes(w: synth.Workload, alpha: float) -> tuple[int, int]:
+    """(active bytes, dense bytes) of one decode step at full caches (pair granularity)."""
+    N = w.seq
+    W = window_table(w.d, w.theta, alpha)
+    a_dec = sum(min(N - 1, x) + 1 for x in W)  # active (key, pair) per (b, kv head)
+    qo = 2 * w.batch * w.q_heads * w.d * 2
+    active = w.batch * w.kv_heads * (4 * a_dec + 2 * w.d * N) + qo
+    dense = w.batch * w.kv_heads * (4 * N * w.d) + qo
+    return active, dense
+
+
+# ------------------------------------------------------------------ measurement helpers
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.rows = []
+        if self.proc is None:
+            return False
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+        return False
+
+    def summary(self):
+        if not getattr(self, "rows", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+def flush_l2(buf):
+    buf.fill_(1)
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def recorded_traffic(kernel_file: str, profile_name: str):
+    """DRAM bytes per launch recorded from an ncu capture, if the kernel source is
+    unchanged since (the profile states the sha256 of the source it measured)."""
+    path = os.path.join(ROOT, "profiles", profile_name)
+    src = os.path.join(ROOT, "rope_frequency_sparse_b200", "csrc", kernel_file)
+    try:
+        text = open(path).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    m_sha = re.search(r"source sha256:\s*([0-9a-f]{64})", text)
+    m_bytes = re.search(r"dram bytes per full-size launch:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_bytes or m_sha.group(1) != sha:
+        return None
+    return float(m_bytes.group(1))
+
+
+# ------------------------------------------------------------------ the timed step
+
+class PrefillStep:
+    """Device-resident inputs and scratch for one windowed prefill step."""
+
+    def __init__(self, w: synth.Workload, seed: int, device):
+        q, k, v = synth.prefill_inputs(w, seed=seed)
+        self.w = w
+        self.host = (q, k, v)
+        self.q, self.k, self.v = q.to(device), k.to(device), v.to(device)
+        self.out = torch.empty_like(self.q)
+        B, S, Hq, d = self.q.shape
+        Hkv = self.k.shape[2]
+        self.ws_bytes = atf.atf_prefill_workspace_bytes(B, S, S, Hq, Hkv, d, atf.ATF_BF16, 0)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
+        self.q_rot = self.ws[: B * S * Hq * d * 2].view(torch.bfloat16).view(B, S, Hq, d)
+        off = ((B * S * Hq * d * 2 + 255) // 256) * 256
+        self.k_rot = self.ws[off: off + B * S * Hkv * d * 2].view(torch.bfloat16).view(B, S, Hkv, d)
+        self.cnt = torch.zeros(1, dtype=torch.int64, device=device)
+
+    def run(self, alpha, stream, ev=None):
+        """RoPE q, RoPE k, windowed prefill: 3 kernel launches.  ev = (e0, e1, e2)
+        brackets the RoPE part and the prefill kernel."""
+        w = self.w
+        B, S, Hq, d = self.q.shape
+        Hkv = self.k.shape[2]
+        if ev:
+            ev[0].record(stream)
+        atf.atf_rope_layout(self.q, self.q_rot, None, B, S, Hq, d, 0, w.theta, 1, atf.ATF_BF16, stream)
+        atf.atf_rope_layout(self.k, self.k_rot, None, B, S, Hkv, d, 0, w.theta, 1, atf.ATF_BF16, stream)
+        if ev:
+            ev[1].record(stream)
+        atf.atf_prefill_ex(self.q_rot, self.k_rot, self.v, self.out, B, S, S, Hq, Hkv, d, 0, atf.ATF_BF16, 1,
+                           w.theta, alpha, self.cnt, None, 0, stream)
+        if ev:
+            ev[2].record(stream)
+
+
+def time_steps(fn, steps, warmup, stream, flush_buf, n_events=3):
+    """Run warmup + steps; per-step CUDA events (the L2 flush between steps is
+    outside the events).  Returns list of per-step event-lists."""
+    for _ in range(warmup):
+        flush_l2(flush_buf)
+        fn(None)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_events)] for _ in range(steps)]
+    for i in range(steps):
+        flush_l2(flush_buf)
+        fn(evs[i])
+    torch.cuda.synchronize()
+    return evs
+
+
+def dist_max(x: float) -> float:
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+    return x
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+def cpu_oracle_sample(w: synth.Workload, alpha: float, target_s: float = 12.0, seed=synth.DEFAULT_SEED):
+    """Time the fp64 oracle on a bounded sample of query rows of the workload."""
+    import oracle  # test infrastructure: the CPU baseline only
+
+    q, k, v = synth.prefill_inputs(w, seed=seed)
+    cores = os.cpu_count() or 1
+    rng = np.random.default_rng(0)
+    n_rows = 8
+    while True:
+        rows = np.sort(rng.choice(w.seq, size=n_rows, replace=False))
+        t0 = time.perf_counter()
+        oracle.prefill(q, k, v, w.theta, alpha, rows=rows, nthreads=cores)
+        dt = time.perf_counter() - t0
+        if dt >= target_s or n_rows >= w.seq:
+            break
+        n_rows = min(w.seq, max(n_rows * 2, int(n_rows * target_s / max(dt, 1e-3))))
+    flops = w.batch * w.q_heads * sum(row_flops(w, alpha, int(m)) for m in rows)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(rows)} random query rows x {w.q_heads} heads of {w.name} (alpha={alpha}); "
+                      f"{dt:.1f} s wall; includes the oracle's one-time fp64 rotation of all keys",
+            "seconds": dt}
+
+
+# ------------------------------------------------------------------ arms
+
+def run_reference(args, rank):
+    """The fp64 CPU oracle as it stands, on this arm's workload and metric."""
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[HEADLINE]
+    vals = []
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, 1.0, target_s=2.0)
+    samples = []
+    for _ in range(args.steps):
+        s = cpu_oracle_sample(w, 1.0, target_s=6.0)
+        vals.append(s["value"])
+        samples.append(s)
+    v = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64)",
+            "config": {"workload": HEADLINE, "batch": 1, "seq_len": w.seq, "q_heads": 28, "kv_heads": 4, "d": 128,
+                       "theta": w.theta, "alpha": 1.0},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": samples[-1]["cores"], "kind": "oracle",
+                             "sample": samples[-1]["sample"]},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream()
+    peaks, peak_kind = measured_peaks()
+    w = synth.WORKLOADS[HEADLINE]
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    step = PrefillStep(w, synth.DEFAULT_SEED + rank, device)
+    s = stream.cuda_stream
+
+    # ---- headline: alpha = 1, timed region bracketed by barrier + sync
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        t_wall = time.perf_counter()
+        evs = time_steps(lambda ev: step.run(1.0, s, ev), args.steps, args.warmup, stream, flush_buf)
+        t_wall = time.perf_counter() - t_wall
+    barrier()
+    torch.cuda.synchronize()
+    atf.atf_check(s)
+    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    kern_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    ms_step = dist_max(sum(step_ms) / len(step_ms))
+    ms_kern = dist_max(sum(kern_ms) / len(kern_ms))
+    eff, dense_flops, skipped = prefill_flops(w, 1.0)
+    value = world * eff / (ms_step * 1e-3) / 1e12
+    cnt_per_step = int(step.cnt.item()) // (args.steps + args.warmup)
+
+    # ---- the same step with every window open (the dense specialisation)
+    evs_d = time_steps(lambda ev: step.run(math.inf, s, ev), args.steps, args.warmup, stream, flush_buf)
+    ms_dense = dist_max(sum(e[0].elapsed_time(e[2]) for e in evs_d) / args.steps)
+    ms_dense_kern = dist_max(sum(e[1].elapsed_time(e[2]) for e in evs_d) / args.steps)
+    per_alpha = {}
+    for a in w.alphas:
+        if a in (1.0,) or math.isinf(a):
+            continue
+        ev_a = time_steps(lambda ev: step.run(a, s, ev), max(3, args.steps // 2), 1, stream, flush_buf)
+        ms_a = sum(e[0].elapsed_time(e[2]) for e in ev_a) / len(ev_a)
+        per_alpha[str(a)] = {"tflops": prefill_flops(w, a)[0] / (ms_a * 1e-3) / 1e12, "ms": ms_a}
+    per_alpha["1.0"] = {"tflops": eff / (ms_step * 1e-3) / 1e12, "ms": ms_step}
+    per_alpha["inf"] = {"tflops": dense_flops / (ms_dense * 1e-3) / 1e12, "ms": ms_dense}
+
+    # ---- end to end through the C ABI from pinned host buffers
+    q_h, k_h, v_h = (t.pin_memory() for t in step.host)
+    out_h = torch.empty_like(q_h).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step(ev):
+        if ev:
+            ev[0].record(stream)
+        step.q.copy_(q_h, non_blocking=True)
+        step.k.copy_(k_h, non_blocking=True)
+        step.v.copy_(v_h, non_blocking=True)
+        B, S, Hq, d = step.q.shape
+        atf.atf_prefill_ex(step.q, step.k, step.v, step.out, B, S, S, Hq, step.k.shape[2], d, 0, atf.ATF_BF16, 0,
+                           w.theta, 1.0, None, step.ws, step.ws_bytes, s)
+        out_h.copy_(step.out, non_blocking=True)
+        if ev:
+            ev[1].record(stream)
+
+    evs_e = time_steps(e2e_step, args.steps, args.warmup, stream, flush_buf, n_events=2)
+    ms_e2e = dist_max(sum(e[0].elapsed_time(e[1]) for e in evs_e) / args.steps)
+    e2e_val = world * eff / (ms_e2e * 1e-3) / 1e12
+
+    extra = {}
+    if world == 1 and not args.no_extra:
+        extra = run_extra(args, device, stream, flush_buf, peaks)
+
+    tflops_kern = eff / (ms_kern * 1e-3) / 1e12
+    traffic = recorded_traffic("prefill_tc.cu", "prefill_tc_layer_8k.md")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded numpy PCG64 N(0,1) -> bf16)",
+        "config": {"workload": HEADLINE, "batch": 1, "seq_len": w.seq, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
+                   "d": w.d, "theta": w.theta, "alpha": 1.0, "parallelism": f"independent layers x{world}",
+                   "l2": "flushed between steps (256 MiB write, outside the per-step CUDA events)"},
+        "speedup_vs_dense": ms_dense / ms_step,
+        "kernel_speedup_vs_dense": ms_dense_kern / ms_kern,
+        "per_alpha": per_alpha,
+        "skipped_pairs_per_step": cnt_per_step, "skipped_pairs_closed_form": skipped,
+        "roofline": {"bound": "tensor", "achieved": tflops_kern, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": tflops_kern / peaks["bf16_tflops"], "traffic": traffic,
+                     "kernel": "prefill_tc_kernel<128,sparse>", "peak_kind": f"{peak_kind} bf16 burst",
+                     "kernel_ms": ms_kern},
+        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": ms_e2e},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(),
+        "wall_s_timed_region": t_wall,
+    }
+    line.update(extra)
+    if world == 1 and rank == 0 and not args.no_cpu:
+        line["cpu_baseline"] = {k2: v2 for k2, v2 in cpu_oracle_sample(w, 1.0).items() if k2 != "seconds"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_extra(args, device, stream, flush_buf, peaks):
+    """Secondary workloads: 32k pair-energy prefill, 128k chunked prefill, 1M-key decode."""
+    s = stream.cuda_stream
+    out = {}
+    # 32k tokens, pair-energy-scaled q/k
+    w3 = synth.WORKLOADS["layer_32k_pair_energy"]
+    st3 = PrefillStep(w3, synth.DEFAULT_SEED, device)
+    ev3 = time_steps(lambda ev: st3.run(1.0, s, ev), 3, 2, stream, flush_buf)
+    ev3d = time_steps(lambda ev: st3.run(math.inf, s, ev), 3, 1, stream, flush_buf)
+    ms3 = sum(e[0].elapsed_time(e[2]) for e in ev3) / 3
+    ms3k = sum(e[1].elapsed_time(e[2]) for e in ev3) / 3
+    ms3d = sum(e[0].elapsed_time(e[2]) for e in ev3d) / 3
+    eff3 = prefill_flops(w3, 1.0)[0]
+    out["layer_32k_pair_energy"] = {"tflops": eff3 / (ms3 * 1e-3) / 1e12, "ms": ms3,
+                                    "kernel_frac_of_peak": eff3 / (ms3k * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                                    "speedup_vs_dense": ms3d / ms3}
+    del st3
+    torch.cuda.empty_cache()
+
+    # 131072 tokens in 16 query chunks of 8192 (keys rotated once into the cache)
+    w4 = synth.WORKLOADS["layer_128k_chunked"]
+    q, k, v = synth.prefill_inputs(w4)
+    qd, kd, vd = q.to(device), k.to(device), v.to(device)
+    del q, k, v
+    B, S, Hq, d = qd.shape
+    Hkv = kd.shape[2]
+    k_rot = torch.empty_like(kd)
+    q_rot = torch.empty((B, w4.q_chunk, Hq, d), dtype=qd.dtype, device=device)
+    o4 = torch.empty_like(qd)
+    C = w4.q_chunk
+
+    def chunked(alpha, ev):
+        if ev:
+            ev[0].record(stream)
+        atf.atf_rope_layout(kd, k_rot, None, B, S, Hkv, d, 0, w4.theta, 1, atf.ATF_BF16, s)
+        for c0 in range(0, S, C):
+            atf.atf_rope_layout(qd[:, c0:c0 + C], q_rot, None, B, C, Hq, d, c0, w4.theta, 1, atf.ATF_BF16, s)
+            atf.atf_prefill_ex(q_rot, k_rot, vd, o4[:, c0:c0 + C], B, C, c0 + C, Hq, Hkv, d, c0, atf.ATF_BF16, 1,
+                               w4.theta, alpha, None, None, 0, s)
+        if ev:
+            ev[1].record(stream)
+
+    res4 = {}
+    for a in (1.0, 0.5, math.inf):
+        ev4 = time_steps(lambda ev: chunked(a, ev), 2, 1, stream, flush_buf, n_events=2)
+        ms4 = sum(e[0].elapsed_time(e[1]) for e in ev4) / 2
+        f4 = prefill_flops(w4, a)[0] if not math.isinf(a) else prefill_flops(w4, a)[1]
+        res4[str(a)] = {"tflops": f4 / (ms4 * 1e-3) / 1e12, "ms": ms4}
+    res4["speedup_vs_dense_alpha1"] = res4["inf"]["ms"] / res4["1.0"]["ms"]
+    out["layer_128k_chunked"] = res4
+    del qd, kd, vd, k_rot, q_rot, o4
+    torch.cuda.empty_cache()
+
+    # decode: 4 sequences x 1,048,576 cached keys (device-generated seeded normals)
+    w5 = synth.WORKLOADS["decode_1m"]
+    g = torch.Generator(device=device)
+    g.manual_seed(synth.DEFAULT_SEED)
+    N = w5.seq
+    kc = torch.randn((w5.batch, w5.kv_heads, w5.d // 16, N, 16), generator=g, device=device).to(torch.bfloat16)
+    v5 = torch.randn((w5.batch, N, w5.kv_heads, w5.d), generator=g, device=device).to(torch.bfloat16)
+    q5 = torch.randn((w5.batch, w5.q_heads, w5.d), generator=g, device=device).to(torch.bfloat16)
+    o5 = torch.empty_like(q5)
+    kv_len = np.full(w5.batch, N, dtype=np.int64)
+    ws_b = atf.atf_decode_workspace_bytes(w5.batch, w5.q_heads, w5.kv_heads, N, w5.d)
+    ws5 = torch.empty(ws_b, dtype=torch.uint8, device=device)
+
+    def dec(alpha, ev):
+        if ev:
+            ev[0].record(stream)
+        atf.atf_decode(q5, kc, v5, o5, w5.batch, kv_len, N, w5.q_heads, w5.kv_heads, w5.d, w5.theta, alpha, ws5,
+                       ws_b, None, s)
+        if ev:
+            ev[1].record(stream)
+
+    ev5 = time_steps(lambda ev: dec(1.0, ev), 10, 3, stream, flush_buf, n_events=2)
+    ev5d = time_steps(lambda ev: dec(math.inf, ev), 10, 3, stream, flush_buf, n_events=2)
+    ms5 = sum(e[0].elapsed_time(e[1]) for e in ev5) / 10
+    ms5d = sum(e[0].elapsed_time(e[1]) for e in ev5d) / 10
+    act, dense_b = decode_bytes(w5, 1.0)
+    gbs = act / (ms5 * 1e-3) / 1e9
+    out["decode_1m"] = {"GBps_active": gbs, "ms": ms5, "ms_dense": ms5d, "speedup_vs_dense": ms5d / ms5,
+                        "active_bytes": act, "dense_bytes": dense_b,
+                        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                     "frac": gbs / peaks["hbm_gbs"],
+                                     "traffic": recorded_traffic("decode.cu", "decode_1m.md")},
+                        "data": "seeded torch CUDA normals (torch.Generator), bf16"}
+    atf.atf_check(s)
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true", help="only the headline workload")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

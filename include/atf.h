@@ -1,0 +1,144 @@
+/*
+ * atf.h -- C ABI of the B200 (sm_100a) library for causal GQA attention with
+ * one distance window per RoPE frequency pair.
+ *
+ * Method: "ATFlash: RoPE-Frequenzen kuerzen Attention-Arbeit um bis zu 57
+ * Prozent" (sudo-ai.de).  Section "Was ATFlash anders macht": RoPE rotates
+ * each frequency pair of q and k; every pair gets its own distance window,
+ * proportional to its wavelength, beyond which its query-key product is left
+ * out, so far keys stay reachable through the slow pairs.  Section "Die Zahlen
+ * - und ihre Grenze": prefill and decode kernels keep the online softmax
+ * unchanged.  This library's reading of "proportional distance":
+ *
+ *   omega_i = theta^(-2i/d),  lambda_i = 2 pi / omega_i,  W_i = ceil(alpha * lambda_i)
+ *   logit(m, n) = (1/sqrt d) * sum_{i : m - n <= W_i} (q~_{2i} k~_{2i} + q~_{2i+1} k~_{2i+1})
+ *   (no active pair -> logit 0, kept in the softmax), then causal softmax and P.V.
+ *   alpha = +infinity gives plain causal RoPE attention.
+ *
+ * Conventions (all entry points):
+ *   - Tensors are dense, row-major, token-major: [batch][token][head][d] with d
+ *     contiguous, unless stated otherwise.  Element type bf16 (ATF_BF16) or
+ *     fp32 (ATF_FP32).  Device pointers must be 16-byte aligned.
+ *   - RoPE pairs are interleaved: pair i = elements (2i, 2i+1); rotation by
+ *     +p*omega_i counter-clockwise for a token at position p.
+ *   - GQA: query head h uses key/value head h / (heads / kv_heads).
+ *   - `stream` is a cudaStream_t (0 = legacy default stream).  Every call is
+ *     asynchronous on it; the return value reports argument and launch errors
+ *     only.  The caller owns every buffer; the library never frees caller
+ *     memory.
+ *   - Supported: d in {64, 128}; heads % kv_heads == 0; heads / kv_heads <= 8
+ *     for decode; theta > 1; alpha > 0 (finite or +inf).
+ *   - Errors: a non-zero atf_status; atf_last_error() gives the message of the
+ *     last failing call on the calling thread.
+ */
+#ifndef ATF_H
+#define ATF_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATF_OK = 0,
+  ATF_ERR_INVALID_ARG = 1, /* null pointer, negative size, inconsistent shape */
+  ATF_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. d = 96) */
+  ATF_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  ATF_ERR_TIMEOUT = 4      /* a kernel's bounded wait expired (see atf_check) */
+} atf_status;
+
+typedef enum { ATF_BF16 = 0, ATF_FP32 = 1 } atf_dtype;
+
+/* Window table.  Writes W_i = ceil(alpha * 2 pi / theta^(-2i/d)), i < d/2, into
+ * the host array W_out (d/2 entries), evaluated in fp64.  alpha = +inf gives
+ * INT64_MAX.  Host only; no GPU needed. */
+atf_status atf_windows(int d, double theta, double alpha, long long* W_out);
+
+/* RoPE + layout (the "RoPE rotates each frequency pair" step of "Was ATFlash
+ * anders macht").
+ *   x:         input  [batch][seq][heads][d], dtype.
+ *   x_rot:     output [batch][seq][heads][d], dtype, may be NULL.  Token t is
+ *              rotated at position pos_offset + t (angles in fp64).
+ *   x_chunked: output [batch][heads][d/16][seq][16] (bf16 only), may be NULL:
+ *              the pair-chunk-major key layout read by atf_decode (chunk c holds
+ *              pairs 8c..8c+7 of every token contiguously).
+ *   rotate:    1 = apply RoPE, 0 = copy / re-layout only (for caches already
+ *              rotated). */
+atf_status atf_rope_layout(const void* x, void* x_rot, void* x_chunked, int batch, int seq, int heads, int d,
+                           long long pos_offset, double theta, int rotate, int dtype, void* stream);
+
+/* Prefill, full form. */
+typedef struct {
+  const void* q;   /* [batch][q_len][heads][d]; query t sits at position q_offset + t */
+  const void* k;   /* [batch][kv_len][kv_heads][d]; key n sits at position n */
+  const void* v;   /* [batch][kv_len][kv_heads][d] */
+  void* out;       /* [batch][q_len][heads][d], same dtype as q */
+  int batch, q_len, kv_len, heads, kv_heads, d;
+  long long q_offset; /* absolute position of query row 0; kv_len >= q_offset + q_len */
+  int dtype;          /* atf_dtype: ATF_BF16 -> tensor-core kernel, ATF_FP32 -> fp32 CUDA-core kernel */
+  int rotated;        /* 1: q and k are already RoPE-rotated (e.g. by atf_rope_layout) */
+  double theta, alpha;
+  unsigned long long* skipped_pairs; /* device, may be NULL: += number of (query head, query,
+                                        key, pair) quadruples outside their window */
+  void* workspace;                   /* device scratch for the rotated q, k when rotated == 0 */
+  size_t workspace_bytes;            /* >= atf_prefill_workspace_bytes(...) when rotated == 0 */
+} atf_prefill_args;
+
+/* Scratch bytes atf_prefill_ex needs for rotated copies of q and k (0 if rotated). */
+size_t atf_prefill_workspace_bytes(int batch, int q_len, int kv_len, int heads, int kv_heads, int d, int dtype,
+                                   int rotated);
+
+/* Prefill (rows a1..a6 of the hot path: windows, RoPE, windowed QK, online
+ * softmax, P.V, epilogue + skip counter).  With alpha = +inf the dense
+ * specialisation of the same kernel runs (no window logic compiled in). */
+atf_status atf_prefill_ex(const atf_prefill_args* args, void* stream);
+
+/* Prefill, short form: batch 1, q_len = kv_len = seq, q_offset 0, bf16,
+ * unrotated q and k.  Scratch for the rotated copies is taken stream-ordered
+ * from the device's default memory pool (cudaMallocAsync / cudaFreeAsync on
+ * `stream`); use atf_prefill_ex with a workspace to avoid that. */
+atf_status atf_prefill(const void* q, const void* k, const void* v, void* out, int seq, int heads, int kv_heads,
+                       int d, double theta, double alpha, void* stream);
+
+/* Decode: one new query per sequence against a rotated key cache.
+ *   q:          [batch][heads][d] bf16, NOT rotated; rotated here at position kv_len[b]-1.
+ *   k_chunked:  [batch][kv_heads][d/16][n_cache][16] bf16, keys already rotated at
+ *               their positions, pair-chunk-major (see atf_rope_layout).
+ *   v:          [batch][n_cache][kv_heads][d] bf16.
+ *   out:        [batch][heads][d] bf16.
+ *   kv_len:     HOST array of batch lengths, 1 <= kv_len[b] <= n_cache; keys
+ *               0..kv_len[b]-1 are live and the query sits at kv_len[b]-1
+ *               (its own key included).
+ *   workspace:  device scratch of >= atf_decode_workspace_bytes(...) bytes
+ *               (split-softmax partials).
+ *   skipped_pairs: device counter, may be NULL (+= skipped (head, key, pair)).
+ * Only the key chunks whose highest pair window still reaches a key are read
+ * from memory; every value row is read. */
+atf_status atf_decode(const void* q, const void* k_chunked, const void* v, void* out, int batch,
+                      const long long* kv_len, long long n_cache, int heads, int kv_heads, int d, double theta,
+                      double alpha, void* workspace, size_t workspace_bytes, unsigned long long* skipped_pairs,
+                      void* stream);
+
+/* Scratch bytes atf_decode needs for `batch` sequences of at most max_kv_len keys. */
+size_t atf_decode_workspace_bytes(int batch, int heads, int kv_heads, long long max_kv_len, int d);
+
+/* Synchronises `stream` and reports ATF_ERR_TIMEOUT if any kernel of this
+ * library on the current device gave up a bounded wait since the last
+ * atf_check (the device error word is cleared), ATF_ERR_CUDA on a CUDA error. */
+atf_status atf_check(void* stream);
+
+/* Failure-detection self test: launches one CTA that waits on a barrier that
+ * nothing ever completes, with a wait limit of `limit_cycles` SM clocks; the
+ * kernel records the expiry in the device error word and returns.  A following
+ * atf_check(stream) returns ATF_ERR_TIMEOUT.  No fault, trap or hang. */
+atf_status atf_selftest_timeout(long long limit_cycles, void* stream);
+
+/* Message of the last failing call on this thread ("" if none). */
+const char* atf_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATF_H */

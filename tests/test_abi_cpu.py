@@ -1,0 +1,108 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+symbol include/atf.h declares, computes the window table like the oracle, and
+rejects bad arguments before touching a device."""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from rope_frequency_sparse_b200 import atf, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return atf.load_library()
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "atf.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(atf_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared_symbols()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+@pytest.mark.parametrize("d,theta", [(64, 1e4), (128, 1e7), (128, 5e5), (64, 1.0001)])
+@pytest.mark.parametrize("alpha", [0.1, 0.5, 1.0, 2.0, math.inf])
+def test_windows_match_oracle(lib, d, theta, alpha):
+    W_lib = atf.atf_windows(d, theta, alpha)
+    W_or, _ = oracle.windows(d, theta, alpha)
+    assert W_lib.tolist() == W_or.tolist()
+
+
+def _status(fn):
+    try:
+        fn()
+    except atf.AtfError as e:
+        return e.status
+    return atf.ATF_OK
+
+
+def test_rejects_bad_arguments_before_any_device_call(lib):
+    fake = 1 << 20  # a 16-byte aligned address; never dereferenced
+    P = atf.atf_prefill_ex
+    assert _status(lambda: P(fake, fake, fake, fake, 1, 128, 128, 28, 4, 96, 0, 0, 1, 1e7, 1.0)) == \
+        atf.ATF_ERR_UNSUPPORTED
+    assert _status(lambda: P(fake, fake, fake, fake, 1, 128, 128, 28, 5, 128, 0, 0, 1, 1e7, 1.0)) == \
+        atf.ATF_ERR_INVALID_ARG
+    assert _status(lambda: P(fake, fake, fake, fake, 1, 128, 100, 28, 4, 128, 0, 0, 1, 1e7, 1.0)) == \
+        atf.ATF_ERR_INVALID_ARG  # kv_len < q_offset + q_len
+    assert _status(lambda: P(None, fake, fake, fake, 1, 128, 128, 28, 4, 128, 0, 0, 1, 1e7, 1.0)) == \
+        atf.ATF_ERR_INVALID_ARG
+    assert _status(lambda: P(fake + 8, fake, fake, fake, 1, 128, 128, 28, 4, 128, 0, 0, 1, 1e7, 1.0)) == \
+        atf.ATF_ERR_INVALID_ARG  # misaligned
+    assert _status(lambda: P(fake, fake, fake, fake, 1, 128, 128, 28, 4, 128, 0, 0, 1, 0.5, 1.0)) == \
+        atf.ATF_ERR_INVALID_ARG  # theta <= 1
+    assert _status(lambda: P(fake, fake, fake, fake, 1, 128, 128, 28, 4, 128, 0, 0, 1, 1e7, -1.0)) == \
+        atf.ATF_ERR_INVALID_ARG  # alpha <= 0
+    assert _status(lambda: P(fake, fake, fake, fake, 1, 128, 128, 28, 4, 128, 0, 0, 0, 1e7, 1.0)) == \
+        atf.ATF_ERR_INVALID_ARG  # unrotated inputs need a workspace
+    assert "workspace" in atf.atf_last_error()
+    D = atf.atf_decode
+    assert _status(lambda: D(fake, fake, fake, fake, 2, [5, 0], 8, 28, 4, 128, 1e7, 1.0, fake, 1 << 20)) == \
+        atf.ATF_ERR_INVALID_ARG  # kv_len 0
+    assert _status(lambda: D(fake, fake, fake, fake, 1, [9], 8, 28, 4, 128, 1e7, 1.0, fake, 1 << 20)) == \
+        atf.ATF_ERR_INVALID_ARG  # kv_len > n_cache
+    assert _status(lambda: D(fake, fake, fake, fake, 1, [8], 8, 36, 4, 128, 1e7, 1.0, fake, 1 << 20)) == \
+        atf.ATF_ERR_UNSUPPORTED  # 9 query heads per kv head
+    assert _status(lambda: D(fake, fake, fake, fake, 1, [8], 8, 28, 4, 128, 1e7, 1.0, fake, 4)) == \
+        atf.ATF_ERR_INVALID_ARG  # workspace too small
+    assert _status(lambda: atf.atf_rope_layout(fake, None, fake, 1, 8, 4, 128, 0, 1e7, 1, atf.ATF_FP32)) == \
+        atf.ATF_ERR_UNSUPPORTED  # chunk-major is bf16 only
+
+
+def test_empty_inputs_are_no_ops(lib):
+    atf.atf_prefill_ex(None, None, None, None, 1, 0, 0, 28, 4, 128, 0, 0, 1, 1e7, 1.0)
+    atf.atf_prefill_ex(None, None, None, None, 0, 16, 16, 28, 4, 128, 0, 0, 1, 1e7, 1.0)
+    atf.atf_decode(None, None, None, None, 0, [], 8, 28, 4, 128, 1e7, 1.0, None, 0)
+    atf.atf_rope_layout(None, None, None, 0, 8, 4, 128, 0, 1e7, 1, 0)
+
+
+def test_workspace_sizes(lib):
+    assert atf.atf_prefill_workspace_bytes(1, 8192, 8192, 28, 4, 128, 0, 1) == 0
+    ws = atf.atf_prefill_workspace_bytes(1, 8192, 8192, 28, 4, 128, 0, 0)
+    assert ws >= 8192 * 28 * 128 * 2 + 8192 * 4 * 128 * 2
+    dws = atf.atf_decode_workspace_bytes(4, 28, 4, 1 << 20, 128)
+    assert dws % (4 * 28 * 130 * 4) == 0 and dws > 0
+
+
+def test_valid_call_without_gpu_fails_loudly(lib):
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    fake = 1 << 20
+    st = _status(lambda: atf.atf_prefill_ex(fake, fake, fake, fake, 1, 128, 128, 28, 4, 128, 0, 0, 1, 1e7, 1.0))
+    assert st == atf.ATF_ERR_CUDA
