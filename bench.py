@@ -278,7 +278,7 @@ def run_ours(args, rank, world, local_rank):
     w = synth.WORKLOADS[HEADLINE]
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     step = PrefillStep(w, synth.DEFAULT_SEED + rank, device)
-    s = stream.cuda_stream
+    s = stream
 
     # ---- headline: alpha = 1, timed region bracketed by barrier + sync
     barrier()
@@ -371,7 +371,7 @@ def run_ours(args, rank, world, local_rank):
 
 def run_extra(args, device, stream, flush_buf, peaks):
     """Secondary workloads: 32k pair-energy prefill, 128k chunked prefill, 1M-key decode."""
-    s = stream.cuda_stream
+    s = stream
     out = {}
     # 32k tokens, pair-energy-scaled q/k
     w3 = synth.WORKLOADS["layer_32k_pair_energy"]

@@ -57,7 +57,7 @@ struct Cfg {
 
 struct Bars {
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full[2], p_full[2], pv_done, q_ready, drain;
+  uint64_t s_full[2], p_full[2], pv_done, o_done, q_ready, drain;
   uint32_t tmem_base;
   int abort;
   int w[kMaxPairs];
@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->p_full[s], 128);
     }
     mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->o_done, 1);
     mbar_init(&bars->q_ready, 128);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -241,6 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&bars->v_empty[s]);
         mma_commit(&bars->pv_done);
+        if (j == T - 1) mma_commit(&bars->o_done);
       }
       if (!ok) {
         mma_commit(&bars->drain);
@@ -406,7 +408,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         corr = ex2_approx(mrun - mnew);
       }
       if (__any_sync(0xffffffffu, need)) {
-        // O holds PV(0..j-1); wait for PV(j-1) before touching it
+        // O holds PV(0..j-1); wait for PV(j-1) before touching it.  PV(j-2) is
+        // known complete (S(j) was issued after it), so pv_done is within one
+        // phase of j-1 and the parity test is exact.
         if (!warp_wait(&bars->pv_done, (j - 1) & 1, abort, p.err, 0x303)) break;
         tc_fence_after();
 #pragma unroll
@@ -440,8 +444,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bars->p_full[j & 1]);
     }
 
-    // ---- epilogue: O / l -> bf16
-    if (j == T && warp_wait(&bars->pv_done, (T - 1) & 1, abort, p.err, 0x304)) {
+    // ---- epilogue: O / l -> bf16.  A one-shot barrier marks the last P.V: a
+    // parity wait on pv_done could be fooled here, since PV(T-2) may still be
+    // pending (two phases outstanding).
+    if (j == T && warp_wait(&bars->o_done, 0, abort, p.err, 0x304)) {
       tc_fence_after();
       const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + q_elem;

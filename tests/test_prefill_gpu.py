@@ -86,7 +86,7 @@ def test_bf16_against_oracle(B, S, Hq, Hkv, d, theta, alpha):
     if not math.isinf(alpha) and S > 200:
         dense, _ = run_gpu(q, k, v, theta, math.inf)
         sparse, _ = run_gpu(q, k, v, theta, alpha)
-        assert np.abs(dense - sparse).max() > 5 * TOL_BF16
+        assert np.abs(dense - sparse).max() > 2 * TOL_BF16
 
 
 def test_bf16_all_pairs_inactive():
