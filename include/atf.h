@@ -123,6 +123,32 @@ atf_status atf_decode(const void* q, const void* k_chunked, const void* v, void*
 /* Scratch bytes atf_decode needs for `batch` sequences of at most max_kv_len keys. */
 size_t atf_decode_workspace_bytes(int batch, int heads, int kv_heads, long long max_kv_len, int d);
 
+/* Decode without any allocation: the same computation as atf_decode, but the
+ * split-softmax partials live in a fixed 8 MiB device array inside the library
+ * instead of a caller workspace.  The pages have no counterpart of this entry
+ * point; it exists for callers that cannot allocate device memory on the decode
+ * path -- a host application whose own memory manager owns all device memory and
+ * forbids allocations behind its back, or a latency-critical serving loop where
+ * an allocation may synchronise the device -- and so cannot hand over a workspace.
+ *   - Arguments as atf_decode, minus the workspace.
+ *   - Fails with ATF_ERR_UNSUPPORTED (no work done) when the call needs more than
+ *     atf_decode_noalloc_scratch_bytes() of scratch, i.e. when
+ *     atf_decode_workspace_bytes(batch, heads, kv_heads, max kv_len, d) is larger.
+ *   - The array is held on every GPU that loads the library until the process
+ *     exits.  The first call on a device looks up its device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *     first call before any stream capture.  It calls no cudaMalloc, cudaFree or
+ *     other allocating routine.
+ *   - All calls on a device share the array and it keeps the previous call's
+ *     contents (every value read is written first in the same call).  Calls whose
+ *     kernels overlap on the GPU (e.g. on unordered streams) race on it. */
+atf_status atf_decode_noalloc(const void* q, const void* k_chunked, const void* v, void* out, int batch,
+                              const long long* kv_len, long long n_cache, int heads, int kv_heads, int d,
+                              double theta, double alpha, unsigned long long* skipped_pairs, void* stream);
+
+/* Size in bytes of atf_decode_noalloc's fixed device scratch array. */
+size_t atf_decode_noalloc_scratch_bytes(void);
+
 /* Synchronises `stream` and reports ATF_ERR_TIMEOUT if any kernel of this
  * library on the current device gave up a bounded wait since the last
  * atf_check (the device error word is cleared), ATF_ERR_CUDA on a CUDA error. */

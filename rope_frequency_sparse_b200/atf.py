@@ -64,6 +64,8 @@ def load_library(path: str = LIB_PATH):
         "atf_prefill": ([vp, vp, vp, vp, i, i, i, i, d, d, vp], i),
         "atf_decode": ([vp, vp, vp, vp, i, vp, ll, i, i, i, d, d, vp, sz, vp, vp], i),
         "atf_decode_workspace_bytes": ([i, i, i, ll, i], sz),
+        "atf_decode_noalloc": ([vp, vp, vp, vp, i, vp, ll, i, i, i, d, d, vp, vp], i),
+        "atf_decode_noalloc_scratch_bytes": ([], sz),
         "atf_check": ([vp], i),
         "atf_selftest_timeout": ([ll, vp], i),
         "atf_last_error": ([], ctypes.c_char_p),
@@ -150,6 +152,19 @@ def atf_decode(q, k_chunked, v, out, batch, kv_len, n_cache, heads, kv_heads, d,
                                      kl.ctypes.data_as(ctypes.c_void_p), int(n_cache), heads, kv_heads, d,
                                      float(theta), float(alpha), _ptr(workspace), int(workspace_bytes),
                                      _ptr(skipped_pairs), _stream(stream)))
+
+
+def atf_decode_noalloc(q, k_chunked, v, out, batch, kv_len, n_cache, heads, kv_heads, d, theta, alpha,
+                       skipped_pairs=None, stream=None):
+    """atf_decode with its scratch in the library's fixed device array (no allocation)."""
+    kl = np.ascontiguousarray(np.asarray(kv_len, dtype=np.int64).reshape(-1))
+    _check(load_library().atf_decode_noalloc(_ptr(q), _ptr(k_chunked), _ptr(v), _ptr(out), batch,
+                                             kl.ctypes.data_as(ctypes.c_void_p), int(n_cache), heads, kv_heads, d,
+                                             float(theta), float(alpha), _ptr(skipped_pairs), _stream(stream)))
+
+
+def atf_decode_noalloc_scratch_bytes() -> int:
+    return int(load_library().atf_decode_noalloc_scratch_bytes())
 
 
 def atf_decode_workspace_bytes(batch, heads, kv_heads, max_kv_len, d) -> int:

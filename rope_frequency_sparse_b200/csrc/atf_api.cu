@@ -145,6 +145,16 @@ __global__ void timeout_selftest_kernel(long long limit, unsigned int* err) {
 
 }  // namespace
 
+atf_status atf::report_error(atf_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
 extern "C" {
 
 const char* atf_last_error(void) { return g_last_error.c_str(); }

@@ -5,6 +5,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "../../include/atf.h"
+
 namespace atf {
 
 constexpr int kMaxPairs = 64;      // d <= 128
@@ -60,6 +62,9 @@ cudaError_t launch_prefill_simt(const PrefillParams& p, cudaStream_t s);
 cudaError_t launch_prefill_tc(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                               bool dense, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
+
+// Records a printf-style message as this thread's atf_last_error() and returns st.
+atf_status report_error(atf_status st, const char* fmt, ...);
 
 // Number of key-range splits per (sequence, kv head) for a decode launch.
 int decode_num_splits(long long max_kv_len, int batch, int hkv);
