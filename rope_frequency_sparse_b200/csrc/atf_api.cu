@@ -105,9 +105,9 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Keys/values [batch][kv_len][kv_heads][d] bf16 as a 4-D tensor (d, head, token,
-// batch); one box = 64 dims x 1 head x 128 tokens, 128-byte swizzle; tokens
-// past kv_len read as zero.
+// A [batch][tokens][heads][d] bf16 tensor (queries, keys or values) as a 4-D
+// tensor (d, head, token, batch); one box = 64 dims x 1 head x 128 tokens,
+// 128-byte swizzle; tokens past the end read as zero.
 atf_status kv_tensor_map(CUtensorMap* map, const void* base, int batch, int kv_len, int hkv, int d) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(ATF_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
@@ -268,10 +268,11 @@ atf_status atf_prefill_ex(const atf_prefill_args* a, void* stream) {
   if (a->dtype == ATF_FP32) {
     e = launch_prefill_simt(p, s);
   } else {
-    CUtensorMap tk, tv;
+    CUtensorMap tq, tk, tv;
+    if (atf_status st = kv_tensor_map(&tq, q, a->batch, a->q_len, a->heads, a->d)) return st;
     if (atf_status st = kv_tensor_map(&tk, k, a->batch, a->kv_len, a->kv_heads, a->d)) return st;
     if (atf_status st = kv_tensor_map(&tv, a->v, a->batch, a->kv_len, a->kv_heads, a->d)) return st;
-    e = launch_prefill_tc(p, tk, tv, std::isinf(a->alpha), s);
+    e = launch_prefill_tc(p, tq, tk, tv, std::isinf(a->alpha), s);
   }
   if (e != cudaSuccess) return cuda_fail(e, "prefill kernel launch");
   return ATF_OK;

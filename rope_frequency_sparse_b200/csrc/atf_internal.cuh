@@ -59,8 +59,8 @@ struct DecodeParams {
 // Launchers (return cudaGetLastError() of the launch).
 cudaError_t launch_rope(const RopeParams& p, cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillParams& p, cudaStream_t s);
-cudaError_t launch_prefill_tc(const PrefillParams& p, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                              bool dense, cudaStream_t s);
+cudaError_t launch_prefill_tc(const PrefillParams& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                              const CUtensorMap& tm_v, bool dense, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
 
 // Records a printf-style message as this thread's atf_last_error() and returns st.
