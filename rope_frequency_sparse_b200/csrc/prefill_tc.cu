@@ -9,33 +9,39 @@
 // recurrence is kept as it is.  Logit: s = (1/sqrt d) sum_{i: Delta <= W_i}
 // (q~_{2i} k~_{2i} + q~_{2i+1} k~_{2i+1}); no active pair gives s = 0.
 //
-// Design (one CTA = 128 query rows of one query head; 10 warps):
-//   warp 0     TMA producer: the Q~ tile once, then K and V tiles of 128 keys
-//              (128B-swizzled boxes of 64 dims) into separate rings.
-//   warp 1     TMEM owner and MMA issuer (one thread):
-//                S(j)  = Q~ . K~(j)^T            A = Q~ tile, B = K tile (both K-major, smem)
-//                O_g  += P(j) . V(j), g = j & 1  A = P in TMEM, B = V tile (MN-major)
-//   warps 2-9  softmax, two groups of four warps; group g takes the KV tiles
-//              j = g, g+2, g+4, ... with one full query row per thread (TMEM
-//              lane = row) and its own running max, row sum and accumulator O_g.
-//              The groups run out of phase, so one group's exponentials overlap
-//              the other group's loads, reductions and corrections; the two
-//              partial results are merged once at the end.
-// TMEM columns: S(j) in buffer j&1 at [128(j&1), 128(j&1)+128) (P(j) is written
-// back over it as packed bf16), O_0 at [256, 256+d), O_1 at [256+d, 256+2d).
+// Design.  One CTA = two Q tiles of 128 query rows (one query head), sharing
+// every K and V tile; 12 warps in three warpgroups:
+//   warp 0      TMA producer: both Q~ tiles once, then K and V tiles of 128 keys
+//               (128B-swizzled boxes of 64 dims) into separate rings.
+//   warp 1      TMEM owner and MMA issuer (one thread), per KV tile j and Q tile g:
+//                 S_g(j)  = Q~_g . K~(j)^T      A = Q~_g (smem), B = K tile (smem)
+//                 O_g    += P_g(j) . V(j)       A = P_g in TMEM, B = V tile (MN-major)
+//   warps 2-3   idle (they complete warpgroup 0 for the register reallocation)
+//   warps 4-7   softmax of Q tile 0, warps 8-11 softmax of Q tile 1: one full
+//               query row per thread (TMEM lane = row), running max, row sum.
+// Warpgroup 0 gives registers to the two softmax warpgroups (setmaxnreg), so a
+// thread holds its whole 128-column row of S at once.
+// TMEM columns: S_g at [128 g, 128 g + 128) (P_g written back over it as packed
+// bf16), O_g at [256 + g d, 256 + (g + 1) d).
+// Issue order: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ... so one Q tile's
+// exponentials overlap the other tile's MMAs.
 //
 // Window structure.  W is non-decreasing in i (wavelengths grow), so the active
 // pairs of any element form a suffix {i >= i*(Delta)}.  KV tiles are visited
-// from the diagonal towards key 0, so the tile's centre distance
-// c_j = m0 - n0_j grows monotonically.  Pairs with W_i < c_j are zeroed in the
-// shared-memory copy of Q~ once and for all, and whole 8-pair chunks below the
-// first non-zeroed pair are not issued to the MMA at all (the contraction depth
-// shrinks tile by tile).  Elements of a tile that straddles a window boundary
-// are fixed on the CUDA cores: a zeroed pair whose window still covers the
-// element is added back, an issued pair whose window does not is subtracted.
-// Each such region is at most half a tile (the side of the boundary away from
-// the tile centre), and only straddling pairs have one.  The per-tile pair
-// ranges are tabulated in shared memory when the CTA starts.
+// from the diagonal towards key 0, so a Q tile's centre distance c = m0 - n0
+// grows monotonically.  Pairs with W_i < c are zeroed in that Q tile's shared-
+// memory copy once and for all, and whole 8-pair chunks below the first
+// non-zeroed pair are not issued to the MMA (the contraction depth shrinks tile
+// by tile).  Elements of a tile that straddles a window boundary are fixed on the
+// CUDA cores before the softmax reads S: a zeroed pair whose window still covers
+// the element is added back, an issued pair whose window does not is subtracted;
+// only straddling pairs, and only 32-column chunks a warp's rows reach, are
+// touched.  The per-tile pair ranges are tabulated in shared memory at the start.
+//
+// Exponentials.  The SFU evaluates 16 ex2 per clock per SM, as many as the
+// tensor core needs cycles for a 128x128 tile's two MMAs, so 3 of every 8 column
+// pairs evaluate 2^x on the FMA pipe instead: x = j + f with j = round(x) and
+// f in [-1/2, 1/2], 2^f by a cubic, j added to the exponent field.
 #include <cuda_bf16.h>
 
 #include "atf_internal.cuh"
@@ -45,33 +51,52 @@ namespace atf {
 
 namespace {
 
-constexpr int BM = 128;        // query rows per CTA
+constexpr int BM = 128;        // query rows per Q tile (MMA M, TMEM lanes)
+constexpr int NQ = 2;          // Q tiles per CTA
 constexpr int BN = 128;        // keys per KV tile
-constexpr int kThreads = 320;  // 10 warps
+constexpr int kThreads = 384;  // 12 warps = 3 warpgroups
+constexpr int kRegsLaunch = 168;   // registers per thread at launch (checked by the launcher)
+constexpr int kRegsCtl = 72;       // warpgroup 0 after reallocation
+constexpr int kRegsSoftmax = 216;  // softmax warpgroups after reallocation
+static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split exceeds the launch");
 constexpr uint32_t kTmemCols = 512;
-constexpr int kTileTable = 1024;  // tabulated KV tiles per CTA (131072 keys)
+constexpr int kStash = 12;        // zeroed query pairs kept per row (more are re-read from global memory)
+constexpr int kTabPairs = 4;      // key pairs converted per batch of boundary corrections
+
+// 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 on [-1/2, 1/2]: coefficients chosen for the
+// smallest maximum relative error (7.5e-5, Lawson's iteratively reweighted least
+// squares in float64, then rounded to float; exp2_poly_fit.py beside the package).
+constexpr float kExpC0 = 0.9999280571937561f;
+constexpr float kExpC1 = 0.6932609677314758f;
+constexpr float kExpC2 = 0.24261093139648438f;
+constexpr float kExpC3 = 0.05517149344086647f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + magic rounds x to an integer
 
 template <int D>
 struct Cfg {
-  static constexpr int NSK = D == 128 ? 3 : 4;   // K ring stages
+  static constexpr int NSK = D == 128 ? 2 : 4;   // K ring stages
   static constexpr int NSV = D == 128 ? 2 : 4;   // V ring stages
   static constexpr int BOXES = D / 64;           // 64-dim swizzle boxes per tile
-  static constexpr int TILE_BYTES = BN * D * 2;  // one K (or V, or Q) tile
+  static constexpr int TILE_BYTES = BN * D * 2;  // one Q, K or V tile
   static constexpr int NCH = D / 16;             // 8-pair chunks = MMA K-steps
   static constexpr int NP = D / 2;
   static constexpr uint32_t COL_S = 0, COL_O = 256;
-  static constexpr int SMEM_TILES = (1 + NSK + NSV) * TILE_BYTES;
+  static constexpr int SMEM_TILES = (NQ + NSK + NSV) * TILE_BYTES;
 };
 
 struct Shared {
-  uint64_t q_full, k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full[2], p_full[2], o_done, q_ready, xfin, drain;
+  uint64_t q_full[NQ], q_ready[NQ], s_full[NQ], p_full[NQ], o_done[NQ];
+  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+  uint64_t drain;
   uint32_t tmem_base;
   int abort;
   int w[kMaxPairs];
-  float fin_m[2][BM];  // per group: running max (log2 units) and row sum, for the final merge
-  float fin_l[2][BM];
-  uint32_t tinfo[kTileTable];  // per KV tile: zeroed | add-back start << 8 | subtract end << 16
+  // Per Q tile, the query pairs most recently zeroed in its shared-memory copy
+  // ([slot][row], slot = pair - first zeroed pair), read back by add-back corrections.
+  uint32_t stash[NQ][kStash][BM];
+  // Per softmax warp: up to kTabPairs key pairs over a 32-column chunk as fp32,
+  // (k_2i(c), k_2i(c+1), k_2i+1(c), k_2i+1(c+1)) per column pair, for the boundary corrections.
+  float4 ktab[8][kTabPairs][16];
 };
 
 template <int D>
@@ -79,35 +104,64 @@ constexpr int smem_bytes() {
   return Cfg<D>::SMEM_TILES + static_cast<int>(sizeof(Shared)) + 1024;
 }
 
-// number of pairs with W_i < x  (W non-decreasing, W_i >= 1)
-__device__ __forceinline__ int lower_bound_w(const int* w, int np, long long x) {
-  int lo = 0, hi = np;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (static_cast<long long>(w[mid]) < x)
-      lo = mid + 1;
-    else
-      hi = mid;
-  }
-  return lo;
-}
+// The rows of one warp (a 32-row quarter q of the Q tile) see, on a KV tile with
+// centre distance `center` (= m0 - n0), the distances Delta = center + 32q + [-127, 31].
+// Their pair ranges:
+//   a: pairs below a lie outside every element's window (W_i < center + 32q - 127)
+//   z: pairs zeroed in these rows of Q~ (W_i < center + 32q + kZeroOffset)
+//   u: pairs from u on lie inside every element's window (W_i >= center + 32q + 31)
+// Pairs in [a, z) are added back where Delta <= W_i, pairs in [z, u) subtracted
+// where Delta > W_i.  kZeroOffset sits near the median distance of a full tile, which
+// keeps both kinds of correction small, and must be <= 1 so that the pairs added
+// back on a tile were zeroed at the step just before it (a(j+1) >= z(j)).
+constexpr int kZeroOffset = -48;
 
-// Pair ranges of a KV tile with centre distance `center` (= m0 - n0):
-//   z: pairs zeroed in Q~ (W_i < center)
-//   a: first pair whose window reaches any element (W_i >= center - 127)
-//   u: end of the pairs whose window misses some element (W_i < center + 127)
-__device__ __forceinline__ uint32_t tile_ranges(const int* w, int np, long long center) {
-  const uint32_t z = lower_bound_w(w, np, center);
-  const uint32_t a = lower_bound_w(w, np, center - (BN - 1));
-  uint32_t u = lower_bound_w(w, np, center + (BM - 1));
-  if (u < z) u = z;
-  return z | (a << 8) | (u << 16);
-}
+// The window table held across a warp: lane l keeps W_l and W_{l+32} (a pair
+// index past the head's pairs holds a sentinel that is never below a threshold).
+struct WarpWindows {
+  long long w0, w1;
+  __device__ __forceinline__ WarpWindows(const int* w, int np, int lane) {
+    w0 = lane < np ? w[lane] : 0x7fffffffffffffffLL;
+    w1 = lane + 32 < np ? w[lane + 32] : 0x7fffffffffffffffLL;
+  }
+  // number of pairs with W_i < x (W is non-decreasing); warp-collective
+  __device__ __forceinline__ int below(long long x) const {
+    return __popc(__ballot_sync(0xffffffffu, w0 < x)) + __popc(__ballot_sync(0xffffffffu, w1 < x));
+  }
+  __device__ __forceinline__ uint32_t quarter_ranges(long long center, int q) const {
+    const long long lo = center + 32 * q;
+    const uint32_t z = below(lo + kZeroOffset);
+    const uint32_t a = below(lo - (BN - 1));
+    const uint32_t u = below(lo + 31);
+    return z | (a << 8) | (u << 16);
+  }
+};
 
 // Byte offset of pair i (4 bytes) of row r inside a 128-row tile stored as
 // 64-dim boxes with the 128-byte swizzle (16-byte chunk index XOR row % 8).
 __device__ __forceinline__ uint32_t pair_offset(int r, int i) {
   return (i >> 5) * (BN * 128) + r * 128 + ((((i & 31) >> 2) ^ (r & 7)) << 4) + (i & 3) * 4;
+}
+
+// Zero the query pairs [lo, hi) of row r in a Q~ tile (swizzled layout above),
+// keeping the old values of pairs lo .. lo+kStash-1 in stash[pair - lo][r].
+// Works on whole 16-byte chunks (4 pairs) of the row.
+__device__ __forceinline__ void zero_pairs(uint8_t* tile, uint32_t (*stash)[BM], int r, int lo, int hi) {
+#pragma unroll 1
+  for (int c4 = lo >> 2; c4 < (hi + 3) >> 2; ++c4) {
+    uint4* p4 = reinterpret_cast<uint4*>(tile + pair_offset(r, 4 * c4));
+    uint4 q = *p4;
+    uint32_t* e = reinterpret_cast<uint32_t*>(&q);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = 4 * c4 + k;
+      if (i >= lo && i < hi) {
+        if (i - lo < kStash) stash[i - lo][r] = e[k];
+        e[k] = 0u;
+      }
+    }
+    *p4 = q;
+  }
 }
 
 // Warp-collective bounded wait: every lane observes the barrier itself (acquire),
@@ -125,6 +179,30 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// 2^x for a pair of floats on the FMA pipe.  x <= 9 here; x is clamped at -126
+// so that the scaled result keeps a valid exponent (2^-126 stands in for 0).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  unpack2(x2, x0, x1);
+  const uint64_t xc = pack2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = fadd2(xc, pack2(kRoundMagic, kRoundMagic));  // low mantissa bits = round(x)
+  const uint64_t f = ffma2(fadd2(t, pack2(-kRoundMagic, -kRoundMagic)), pack2(-1.f, -1.f), xc);
+  uint64_t q = ffma2(pack2(kExpC3, kExpC3), f, pack2(kExpC2, kExpC2));
+  q = ffma2(q, f, pack2(kExpC1, kExpC1));
+  q = ffma2(q, f, pack2(kExpC0, kExpC0));
+  float q0, q1, t0, t1;
+  unpack2(q, q0, q1);
+  unpack2(t, t0, t1);
+  // (bits(t) << 23) == round(x) << 23 modulo 2^32: the magic's own bits shift out
+  return pack2(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+               __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
+}
+
+// column pairs k (columns 2k, 2k+1) whose exponentials use the FMA pipe
+__host__ __device__ constexpr bool exp_on_fma(int k) {
+  return (k & 7) == 1 || (k & 7) == 4 || (k & 7) == 6;
+}
+
 }  // namespace
 
 template <int D, bool SPARSE>
@@ -135,50 +213,54 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NSK = C::NSK, NSV = C::NSV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                      // Q~ tile
-  uint8_t* sK = smem + C::TILE_BYTES;      // [NSK][TILE_BYTES]
+  uint8_t* sQ = smem;                      // [NQ][TILE_BYTES]
+  uint8_t* sK = sQ + NQ * C::TILE_BYTES;   // [NSK][TILE_BYTES]
   uint8_t* sV = sK + NSK * C::TILE_BYTES;  // [NSV][TILE_BYTES]
   Shared* sh = reinterpret_cast<Shared*>(smem + C::SMEM_TILES);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // ---- tile coordinates: heaviest query tiles first
+  // ---- coordinates: Q tiles 2 pr and 2 pr + 1 of one (batch, head); heaviest CTAs first
   const int nqt = (p.q_len + BM - 1) / BM;
+  const int npr = (nqt + NQ - 1) / NQ;
   int idx = blockIdx.x;
   const int h = idx % p.hq;
   idx /= p.hq;
   const int b = idx % p.batch;
-  const int qt = nqt - 1 - idx / p.batch;
+  const int pr = npr - 1 - idx / p.batch;
   const int hk = h / (p.hq / p.hkv);
-  const long long m0 = p.q_offset + static_cast<long long>(qt) * BM;
-  const int rows_here = min(BM, p.q_len - qt * BM);
-  const long long max_key = min(m0 + rows_here - 1, static_cast<long long>(p.kv_len) - 1);
-  const int T = static_cast<int>(max_key / BN) + 1;  // KV tiles, visited j = 0..T-1
+  const int t0 = pr * NQ * BM;             // first query row of the CTA
+  const long long m0 = p.q_offset + t0;    // its position
+  const int rows1 = max(0, min(BM, p.q_len - t0 - BM));
+  const int nq = rows1 > 0 ? 2 : 1;        // Q tiles with rows
+  const long long kv_last = static_cast<long long>(p.kv_len) - 1;
+  const long long maxkey0 = min(m0 + min(BM, p.q_len - t0) - 1, kv_last);
+  const long long maxkey = nq == 2 ? min(m0 + BM + rows1 - 1, kv_last) : maxkey0;
+  const int T = static_cast<int>(maxkey / BN) + 1;              // KV tiles, visited j = 0..T-1
+  const int jstart0 = T - 1 - static_cast<int>(maxkey0 / BN);  // Q tile 0 starts one tile later or not
+  auto jstart = [&](int g) { return g == 0 ? jstart0 : 0; };
   auto tile_n0 = [&](int j) { return static_cast<long long>(T - 1 - j) * BN; };
-  auto ranges = [&](int j) -> uint32_t {
-    if (!SPARSE) return 0u;
-    if (j < kTileTable) return sh->tinfo[j];
-    return tile_ranges(sh->w, C::NP, m0 - tile_n0(j));
-  };
+  // Q tile g on KV tile j has centre m0 + 128 g - n0(j) = m0 - n0(j + g): entry j + g.
+  auto centre = [&](int e) { return m0 - static_cast<long long>(T - 1 - e) * BN; };
+
 
   // ---- setup
   if (tid == 0) {
-    mbar_init(&sh->q_full, 1);
+    for (int g = 0; g < NQ; ++g) {
+      mbar_init(&sh->q_full[g], 1);
+      mbar_init(&sh->q_ready[g], 128);
+      mbar_init(&sh->s_full[g], 1);
+      mbar_init(&sh->p_full[g], 128);
+      mbar_init(&sh->o_done[g], 1);
+    }
     for (int s = 0; s < NSK; ++s) {
       mbar_init(&sh->k_full[s], 1);
-      mbar_init(&sh->k_empty[s], 4);
+      mbar_init(&sh->k_empty[s], 8);  // every softmax warp, once per KV tile
     }
     for (int s = 0; s < NSV; ++s) {
       mbar_init(&sh->v_full[s], 1);
       mbar_init(&sh->v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sh->s_full[s], 1);
-      mbar_init(&sh->p_full[s], 128);
-    }
-    mbar_init(&sh->o_done, 1);
-    mbar_init(&sh->q_ready, 128);
-    mbar_init(&sh->xfin, 256);
     mbar_init(&sh->drain, 1);
     sh->abort = 0;
     fence_mbar_init();
@@ -194,23 +276,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_v);
   }
   __syncthreads();
-  if (SPARSE) {
-    const int nt = T < kTileTable ? T : kTileTable;
-    for (int j = tid; j < nt; j += kThreads) sh->tinfo[j] = tile_ranges(sh->w, C::NP, m0 - tile_n0(j));
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
   volatile int* abort = &sh->abort;
 
-  if (warp == 0) {
-    // ================================================================ TMA producer
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&sh->q_full, C::TILE_BYTES);
+  if (warp < 4) {
+    setmaxnreg_dec<kRegsCtl>();
+    if (warp == 0 && lane == 0) {
+      // ============================================================== TMA producer
+      for (int g = 0; g < nq; ++g) {
+        mbar_arrive_expect_tx(&sh->q_full[g], C::TILE_BYTES);
 #pragma unroll
-      for (int bx = 0; bx < C::BOXES; ++bx)
-        tma_load_4d(sQ + bx * (BN * 128), &tm_q, &sh->q_full, bx * 64, h, qt * BM, b);
+        for (int bx = 0; bx < C::BOXES; ++bx)
+          tma_load_4d(sQ + g * C::TILE_BYTES + bx * (BN * 128), &tm_q, &sh->q_full[g], bx * 64, h, t0 + g * BM, b);
+      }
       int k_issued = 0, v_issued = 0;
       for (int j = 0; j < T; ++j) {
         const int n0 = static_cast<int>(tile_n0(j));
@@ -235,319 +316,398 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (*abort) {
         // let every load already issued land before the CTA leaves
-        drain_wait(&sh->q_full, 0);
+        for (int g = 0; g < nq; ++g) drain_wait(&sh->q_full[g], 0);
         for (int j = 0; j < k_issued; ++j) drain_wait(&sh->k_full[j % NSK], (j / NSK) & 1);
         for (int j = 0; j < v_issued; ++j) drain_wait(&sh->v_full[j % NSV], (j / NSV) & 1);
       }
-    }
-  } else if (warp == 1) {
-    // ================================================================ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 1) {
+      // ============================================================== MMA issuer
+      // The whole warp runs the loop (warp-uniform descriptors and waits); one
+      // elected lane, always the same one, issues the MMAs and their commits.
       constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, false, true);
-      constexpr uint64_t kdesc_bits = smem_desc_bits(16, 1024, kLayoutSW128);
-      constexpr uint64_t vdesc_bits = smem_desc_bits(BN * 128, 1024, kLayoutSW128);
-      const uint32_t sQ_addr = smem_u32(sQ), sK_addr = smem_u32(sK), sV_addr = smem_u32(sV);
-      int ev = 0;
-      bool ok = mbar_wait(&sh->q_ready, ev & 1, abort, p.err, 0x201);
-      ++ev;
+      constexpr uint64_t kTileStep = C::TILE_BYTES >> 4;  // descriptor address units
+      const uint64_t dq0 = smem_desc(smem_u32(sQ), smem_desc_bits(16, 1024, kLayoutSW128));
+      const uint64_t dk0 = smem_desc(smem_u32(sK), smem_desc_bits(16, 1024, kLayoutSW128));
+      const uint64_t dv0 = smem_desc(smem_u32(sV), smem_desc_bits(BN * 128, 1024, kLayoutSW128));
+      const WarpWindows ww(sh->w, C::NP, lane);
+      bool ok = true;
+      for (int g = 0; ok && g < nq; ++g) ok = warp_wait(&sh->q_ready[g], 0, abort, p.err, 0x201);
       tc_fence_after();
-      auto issue_s = [&](int j) -> bool {
+      int k_seen = 0;  // K tiles whose arrival this thread has observed
+      auto issue_s = [&](int g, int j) -> bool {
         const int s = j % NSK;
-        if (!mbar_wait(&sh->k_full[s], (j / NSK) & 1, abort, p.err, 0x202)) return false;
-        tc_fence_after();
-        const int c0 = static_cast<int>(ranges(j) & 0xFF) >> 3;
-        const uint32_t d_tmem = tmem + C::COL_S + (j & 1) * BN;
-        for (int c = c0; c < C::NCH; ++c) {
-          const uint32_t koff = (c >> 2) * (BN * 128) + (c & 3) * 32;
-          mma_ss(d_tmem, smem_desc(sQ_addr + koff, kdesc_bits),
-                 smem_desc(sK_addr + s * C::TILE_BYTES + koff, kdesc_bits), idesc_qk, c > c0 ? 1u : 0u);
+        if (j >= k_seen) {
+          if (!warp_wait(&sh->k_full[s], (j / NSK) & 1, abort, p.err, 0x202)) return false;
+          k_seen = j + 1;
+          tc_fence_after();
         }
-        mma_commit(&sh->s_full[j & 1]);
+        // pairs zeroed in every row of Q~_g (those of its first quarter): chunks below are skipped
+        const int c0 = SPARSE ? ww.below(centre(j + g) + kZeroOffset) >> 3 : 0;
+        const uint32_t d_tmem = tmem + C::COL_S + g * BN;
+        const uint64_t aq = dq0 + g * kTileStep, bk = dk0 + s * kTileStep;
+        if (elect_one()) {
+#pragma unroll
+          for (int c = 0; c < C::NCH; ++c) {
+            const uint64_t off = static_cast<uint64_t>((c >> 2) * (BN * 128) + (c & 3) * 32) >> 4;
+            if (SPARSE)
+              mma_ss_if(d_tmem, aq + off, bk + off, idesc_qk, c > c0 ? 1u : 0u, c >= c0 ? 1u : 0u);
+            else
+              mma_ss(d_tmem, aq + off, bk + off, idesc_qk, c > 0 ? 1u : 0u);
+          }
+          mma_commit(&sh->s_full[g]);
+        }
+        __syncwarp();
         return true;
       };
-      if (ok) ok = issue_s(0);
+      for (int g = 0; ok && g < nq; ++g)
+        if (jstart(g) == 0) ok = issue_s(g, 0);
       for (int j = 0; ok && j < T; ++j) {
-        if (j + 1 < T) {
-          if (SPARSE && (ranges(j + 1) & 0xFF) > (ranges(j) & 0xFF)) {
-            ok = mbar_wait(&sh->q_ready, ev & 1, abort, p.err, 0x203);
-            ++ev;
-            if (!ok) break;
+        const int sv = j % NSV;
+        bool v_seen = false;
+        for (int g = 0; g < nq; ++g) {
+          if (j >= jstart(g)) {
+            if (!v_seen) {
+              if (!(ok = warp_wait(&sh->v_full[sv], (j / NSV) & 1, abort, p.err, 0x205))) break;
+              v_seen = true;
+            }
+            if (!(ok = warp_wait(&sh->p_full[g], (j - jstart(g)) & 1, abort, p.err, 0x204))) break;
             tc_fence_after();
-          }
-          // S(j+1) overwrites the TMEM buffer that holds P(j-1); PV(j-1) was issued
-          // before it by this thread, and tcgen05.mma operations execute in issue order.
-          if (!(ok = issue_s(j + 1))) break;
-        }
-        const int s = j % NSV;
-        // V(j) normally landed long ago: check it before blocking on P(j)
-        if (!(ok = mbar_wait(&sh->v_full[s], (j / NSV) & 1, abort, p.err, 0x205))) break;
-        if (!(ok = mbar_wait(&sh->p_full[j & 1], (j >> 1) & 1, abort, p.err, 0x204))) break;
-        tc_fence_after();
-        const uint32_t p_tmem = tmem + C::COL_S + (j & 1) * BN;  // P(j) packed bf16 over S(j)
-        const uint32_t o_tmem = tmem + C::COL_O + (j & 1) * D;   // this group's accumulator
+            const uint32_t p_tmem = tmem + C::COL_S + g * BN;  // P_g(j), packed bf16 over S_g(j)
+            const uint32_t o_tmem = tmem + C::COL_O + g * D;
+            const uint64_t bv = dv0 + sv * kTileStep;
+            const bool first = j == jstart(g);
+            if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint32_t a = sV_addr + s * C::TILE_BYTES + kk * 2048;
-          mma_ts(o_tmem, p_tmem + 8 * kk, smem_desc(a, vdesc_bits), idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < BN / 16; ++kk)
+                mma_ts(o_tmem, p_tmem + 8 * kk, bv + ((kk * 2048) >> 4), idesc_pv, (!first || kk > 0) ? 1u : 0u);
+              if (j == T - 1) mma_commit(&sh->o_done[g]);
+            }
+            __syncwarp();
+          }
+          // S_g(j+1) overwrites P_g(j); PV_g(j) was issued first and tcgen05.mma
+          // operations of one thread execute in issue order.
+          if (j + 1 < T && j + 1 >= jstart(g) && !(ok = issue_s(g, j + 1))) break;
         }
-        mma_commit(&sh->v_empty[s]);
-        if (j == T - 1) mma_commit(&sh->o_done);
+        if (!ok) break;
+        if (elect_one()) mma_commit(&sh->v_empty[sv]);
+        __syncwarp();
       }
       if (!ok) {
-        mma_commit(&sh->drain);
+        if (elect_one()) mma_commit(&sh->drain);
+        __syncwarp();
         drain_wait(&sh->drain, 0);
       }
     }
   } else {
-    // ================================================================ softmax (warps 2..9)
-    const int quarter = warp & 3;
-    const int g = (warp - 2) >> 2;      // group: KV tiles j with j % 2 == g
-    const int r = quarter * 32 + lane;  // query row in tile == TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const int t = qt * BM + r;
-    const bool row_ok = t < p.q_len;
-    const long long m = m0 + r;
-    const long long q_elem = ((static_cast<long long>(b) * p.q_len + (row_ok ? t : 0)) * p.hq + h) * D;
-    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(p.q) + q_elem);
-    constexpr float kLog2e = 1.4426950408889634f;
-    const float scale = kLog2e * rsqrtf(static_cast<float>(D));
+    setmaxnreg_inc<kRegsSoftmax>();
+    // ================================================================ softmax (warps 4..11)
+    const int g = (warp - 4) >> 2;      // Q tile
+    const int quarter = warp & 3;       // TMEM lanes 32*quarter.. of this warp
+    const int r = quarter * 32 + lane;  // query row in the tile == TMEM lane
+    const WarpWindows ww(sh->w, C::NP, lane);
+    if (g >= nq) {
+      // no rows in this Q tile: only keep the K ring's release count
+      for (int j = 0; j < T; ++j) {
+        if (!warp_wait(&sh->k_full[j % NSK], (j / NSK) & 1, abort, p.err, 0x300)) break;
+        if (lane == 0) mbar_arrive(&sh->k_empty[j % NSK]);
+      }
+    } else {
+      uint8_t* sQg = sQ + g * C::TILE_BYTES;
+      const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+      const uint32_t s_tmem = tmem + lane_off + C::COL_S + g * BN;
+      const int t = t0 + g * BM + r;
+      const bool row_ok = t < p.q_len;
+      const long long m = m0 + g * BM + r;
+      const long long q_elem = ((static_cast<long long>(b) * p.q_len + (row_ok ? t : 0)) * p.hq + h) * D;
+      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(p.q) + q_elem);
+      constexpr float kLog2e = 1.4426950408889634f;
+      const float scale = kLog2e * rsqrtf(static_cast<float>(D));
+      const int j0 = jstart(g);
 
-    bool ok = true;
-    // Pairs dead in the first tile are zeroed in the Q~ tile before S(0).
-    if (g == 0) {
-      ok = warp_wait(&sh->q_full, 0, abort, p.err, 0x300);
+      bool ok = warp_wait(&sh->q_full[g], 0, abort, p.err, 0x301);
       if (ok) {
-        if (SPARSE) {
-          const int z0 = static_cast<int>(ranges(0) & 0xFF);
-          for (int i = 0; i < z0; ++i) *reinterpret_cast<uint32_t*>(sQ + pair_offset(r, i)) = 0u;
+        if (SPARSE) {  // pairs dead in this Q tile's first KV tile
+          const int z0 = static_cast<int>(ww.quarter_ranges(centre(j0 + g), quarter) & 0xFF);
+          zero_pairs(sQg, sh->stash[g], r, 0, z0);
           fence_proxy_async_smem();
         }
-        mbar_arrive(&sh->q_ready);
+        mbar_arrive(&sh->q_ready[g]);
       }
-    }
+      for (int j = 0; ok && j < j0; ++j) {  // KV tiles entirely after this Q tile's rows
+        if ((ok = warp_wait(&sh->k_full[j % NSK], (j / NSK) & 1, abort, p.err, 0x302)) && lane == 0)
+          mbar_arrive(&sh->k_empty[j % NSK]);
+      }
 
-    float mrun = -INFINITY;
-    uint64_t lsum2 = 0ull;  // packed partial row sums
-    unsigned long long cnt = 0;
-    for (int j = g; ok && j < T; j += 2) {
-      const int s = j % NSK;
-      const long long n0 = tile_n0(j);
-      const long long center = m0 - n0;
-      const uint32_t rg = ranges(j);
-      const int z = static_cast<int>(rg & 0xFF);
-      const int a = static_cast<int>((rg >> 8) & 0xFF);
-      const int u = static_cast<int>((rg >> 16) & 0xFF);
-      // prefetch the query pairs of this tile's first boundary corrections
-      uint32_t qpf[4] = {0u, 0u, 0u, 0u};
-      if (SPARSE && row_ok) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if (a + k < u) qpf[k] = __ldg(qrow + a + k);
-      }
-      if (!(ok = warp_wait(&sh->s_full[j & 1], (j >> 1) & 1, abort, p.err, 0x301))) break;
-      tc_fence_after();
-      if (SPARSE && j + 1 < T) {
-        const int zn = static_cast<int>(ranges(j + 1) & 0xFF);
-        if (zn > z) {  // S(j) is done reading Q~: zero the newly dead pairs for S(j+1)
-          for (int i = z; i < zn; ++i) *reinterpret_cast<uint32_t*>(sQ + pair_offset(r, i)) = 0u;
-          fence_proxy_async_smem();
-          mbar_arrive(&sh->q_ready);
-        }
-      }
-      const uint32_t s_tmem = tmem + lane_off + C::COL_S + (j & 1) * BN;
-      const bool has_mma = (z >> 3) < C::NCH;  // a tile whose pairs are all zeroed has no S MMA
-      // valid columns of this row form the prefix [0, cmax]
-      int cmax = -1;
-      if (row_ok) {
-        long long cmx = min(static_cast<long long>(BN - 1), m - n0);
-        cmx = min(cmx, static_cast<long long>(p.kv_len) - 1 - n0);
-        cmax = static_cast<int>(cmx);
-      }
-      const bool partial = __any_sync(0xffffffffu, cmax < BN - 1);
-      // ---- pass 1 over S in chunks of 64 columns: boundary corrections (written
-      // back to TMEM) and the row max (eight independent 3-input max chains)
-      float acc[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) acc[k] = -INFINITY;
-      bool stored = false;
-      // the K tile is read only by boundary corrections
-      if (SPARSE && a < u && !(ok = warp_wait(&sh->k_full[s], (j / NSK) & 1, abort, p.err, 0x302))) break;
-      if (SPARSE) {
-        const int nv = cmax + 1;  // valid columns of this row
-        cnt += static_cast<unsigned long long>(a) * nv;
-        for (int i = a; i < u; ++i) {
-          const long long tl = r + center - sh->w[i];
-          const int tli = static_cast<int>(tl < -1 ? -1 : (tl > BN ? BN : tl));
-          cnt += static_cast<unsigned long long>(tli <= 0 ? 0 : (tli < nv ? tli : nv));
-        }
-      }
-#pragma unroll
-      for (int hc = 0; hc < 2; ++hc) {
-        float v[64];
-        if (has_mma) {
-          tmem_ld32(s_tmem + 64 * hc, reinterpret_cast<uint32_t*>(v));
-          tmem_ld32(s_tmem + 64 * hc + 32, reinterpret_cast<uint32_t*>(v + 32));
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) v[c] = 0.f;
-        }
+      float mrun = -INFINITY;
+      uint64_t lsum2 = 0ull;  // packed partial row sums
+      unsigned long long cnt = 0;
+      int zst = 0;  // first pair held in this warp's rows of the stash
+      uint32_t qr = SPARSE ? ww.quarter_ranges(centre(j0 + g), quarter) : 0u;
+      for (int j = j0; ok && j < T; ++j) {
+        const int s = j % NSK;
+        const long long n0 = tile_n0(j);
+        const long long center = m0 + g * BM - n0;
+        const int z = static_cast<int>(qr & 0xFF);
+        const int a = static_cast<int>((qr >> 8) & 0xFF);
+        const int u = static_cast<int>((qr >> 16) & 0xFF);
+        // the next tile's ranges, computed while S is still on its way
+        const uint32_t qr_next = (SPARSE && j + 1 < T) ? ww.quarter_ranges(center + BN, quarter) : 0u;
+        if (!(ok = warp_wait(&sh->s_full[g], (j - j0) & 1, abort, p.err, 0x303))) break;
+        tc_fence_after();
+        // valid columns of this row form the prefix [0, cmax]
+        int cmax = -1;
+        if (row_ok) cmax = static_cast<int>(min(static_cast<long long>(BN - 1), min(m, kv_last) - n0));
+        const bool partial = __any_sync(0xffffffffu, cmax < BN - 1);
+        // no S MMA when every pair is zeroed in every row
+        const bool has_mma = !SPARSE || (ww.below(center + kZeroOffset) >> 3) < C::NCH;
+        uint32_t s_chunks = has_mma ? 0xFu : 0u;  // 32-column chunks of S held in TMEM
         if (SPARSE) {
-          bool touched = !has_mma;  // a tile without S MMA must write its (zero) logits
-          const uint32_t kbase = smem_u32(sK + s * C::TILE_BYTES);
-          for (int i = a; i < u; ++i) {
-            const int wi = sh->w[i];
-            const long long tl = r + center - wi;             // columns c < tl are outside pair i's window
-            const long long tw = quarter * 32 + center - wi;  // smallest tl of the warp
-            const int tli = static_cast<int>(tl < -1 ? -1 : (tl > BN ? BN : tl));
-            const bool add = i < z;  // zeroed pair: add back where c >= tl; else subtract where c < tl
-            // skip this chunk when no row of the warp has an element of it on the corrected side
-            if (add ? (64 * hc + 63 < tw) : (64 * hc >= tw + 31)) continue;
-            touched = true;
-            const int kq = i - a;
-            const uint32_t qp = kq == 0   ? qpf[0]
-                                : kq == 1 ? qpf[1]
-                                : kq == 2 ? qpf[2]
-                                : kq == 3 ? qpf[3]
-                                          : (row_ok ? __ldg(qrow + i) : 0u);
-            const float qa = bf16lo_to_f32(qp), qb = bf16hi_to_f32(qp);
-            const float sg = add ? 1.f : -1.f;
-            uint32_t xo[8];
-            {
-              const uint32_t base = kbase + (i >> 5) * (BN * 128) + (i & 3) * 4;
-              const uint32_t ch = (i & 31) >> 2;
+          const int nv = cmax + 1;  // valid columns of this row
+          cnt += static_cast<unsigned long long>(a) * nv;
+          if (__builtin_expect(a < u, 0)) {
+            // ---- boundary corrections, in place on S in TMEM, 32 columns at a time.
+            // For pairs in [a, u) the windows lie within 127 of the centre, so the
+            // thresholds fit in 32 bits.
+            const int cen = static_cast<int>(center);
+            const int cw = quarter * 32 + cen;  // threshold offset of the warp's first row
+            const uint32_t kbase = smem_u32(sK + s * C::TILE_BYTES);
+#pragma unroll 1
+            for (int hb = a; hb < u; hb += 32) {
+              // classify pair hb + lane: the chunks some row of this warp must
+              // correct (tm), and those every row corrects entirely (fm)
+              const int il = hb + lane;
+              const bool valid = il < u;
+              const int wl = valid ? sh->w[il] : 0;
+              const int twl = cw - wl;  // smallest threshold among the warp's rows
+              const bool addl = il < z;
+              uint32_t tm = 0u, fm = 0u;
 #pragma unroll
-              for (int x = 0; x < 8; ++x) xo[x] = base + ((ch ^ x) << 4);
-            }
+              for (int qc = 0; qc < BN / 32; ++qc) {
+                const int c_lo = 32 * qc;
+                const bool touch = valid && (addl ? (c_lo + 31 >= twl) : (c_lo < twl + 31));
+                const bool fullc = valid && (addl ? (c_lo >= twl + 31) : (c_lo + 31 < twl));
+                tm |= static_cast<uint32_t>(touch) << qc;
+                fm |= static_cast<uint32_t>(fullc) << qc;
+              }
+#pragma unroll 1
+              for (int qc = 0; qc < BN / 32; ++qc) {
+                const int c_lo = 32 * qc;
+                uint32_t tbits = __ballot_sync(0xffffffffu, (tm >> qc) & 1u);
+                const uint32_t fbits = __ballot_sync(0xffffffffu, (fm >> qc) & 1u);
+                if (!tbits) continue;
+                float x[32];
+                if ((s_chunks >> qc) & 1u) {
+                  tmem_ld32(s_tmem + c_lo, reinterpret_cast<uint32_t*>(x));
+                  tmem_ld_wait();
+                } else {
 #pragma unroll
-            for (int cc = 0; cc < 64; ++cc) {
-              const int c = 64 * hc + cc;
-              const uint32_t kp = lds32(xo[cc & 7] + c * 128);
-              const float pd = fmaf(qa, bf16lo_to_f32(kp), qb * bf16hi_to_f32(kp));
-              const bool inside = add ? (c >= tli) : (c < tli);
-              v[cc] = inside ? fmaf(sg, pd, v[cc]) : v[cc];
+                  for (int cc = 0; cc < 32; ++cc) x[cc] = 0.f;
+                }
+                do {
+                  // up to kTabPairs pairs: convert their keys for this chunk, then apply
+                  int kb[kTabPairs];
+                  uint32_t qpb[kTabPairs];
+                  int nb = 0;
+#pragma unroll
+                  for (int b = 0; b < kTabPairs; ++b) {
+                    kb[b] = 0;
+                    qpb[b] = 0u;
+                    if (tbits) {  // warp-uniform
+                      const int k = __ffs(tbits) - 1;
+                      tbits &= tbits - 1;
+                      kb[b] = k;
+                      nb = b + 1;
+                      const int i = hb + k;
+                      const uint32_t kw = lds32(kbase + (i >> 5) * (BN * 128) + (i & 3) * 4 + (c_lo + lane) * 128 +
+                                                ((((i & 31) >> 2) ^ (lane & 7)) << 4));
+                      const uint32_t kn = __shfl_down_sync(0xffffffffu, kw, 1);
+                      if (!(lane & 1))
+                        sh->ktab[warp - 4][b][lane >> 1] =
+                            make_float4(bf16lo_to_f32(kw), bf16lo_to_f32(kn), bf16hi_to_f32(kw), bf16hi_to_f32(kn));
+                      if (row_ok) {
+                        if (i >= z)
+                          qpb[b] = *reinterpret_cast<const uint32_t*>(sQg + pair_offset(r, i));
+                        else if (static_cast<unsigned>(i - zst) < static_cast<unsigned>(kStash))
+                          qpb[b] = sh->stash[g][i - zst][r];
+                        else
+                          qpb[b] = __ldg(qrow + i);
+                      }
+                    }
+                  }
+                  __syncwarp();
+#pragma unroll 1
+                  for (int b = 0; b < nb; ++b) {
+                    const int k = b == 0 ? kb[0] : b == 1 ? kb[1] : b == 2 ? kb[2] : kb[3];
+                    const uint32_t qp = b == 0 ? qpb[0] : b == 1 ? qpb[1] : b == 2 ? qpb[2] : qpb[3];
+                    const int i = hb + k;
+                    const int wi = __shfl_sync(0xffffffffu, wl, k);
+                    const bool add = i < z;  // zeroed pair: add back where c >= tl; else subtract where c < tl
+                    const float sg = add ? 1.f : -1.f;
+                    const uint64_t qa2 = pack2(sg * bf16lo_to_f32(qp), sg * bf16lo_to_f32(qp));
+                    const uint64_t qb2 = pack2(sg * bf16hi_to_f32(qp), sg * bf16hi_to_f32(qp));
+                    const float4* tab = sh->ktab[warp - 4][b];
+                    if ((fbits >> k) & 1u) {  // every row of the warp corrects the whole chunk
+#pragma unroll
+                      for (int cp = 0; cp < 16; ++cp) {
+                        const float4 t = tab[cp];
+                        uint64_t x2 = pack2(x[2 * cp], x[2 * cp + 1]);
+                        x2 = ffma2(qa2, pack2(t.x, t.y), x2);
+                        x2 = ffma2(qb2, pack2(t.z, t.w), x2);
+                        unpack2(x2, x[2 * cp], x[2 * cp + 1]);
+                      }
+                    } else {
+                      const int tc = r + cen - wi - c_lo;  // chunk columns cc < tc lie outside the window
+#pragma unroll
+                      for (int cp = 0; cp < 16; ++cp) {
+                        const float4 t = tab[cp];
+                        uint64_t y2 = pack2(x[2 * cp], x[2 * cp + 1]);
+                        y2 = ffma2(qa2, pack2(t.x, t.y), y2);
+                        y2 = ffma2(qb2, pack2(t.z, t.w), y2);
+                        float y0, y1;
+                        unpack2(y2, y0, y1);
+                        if ((2 * cp >= tc) == add) x[2 * cp] = y0;
+                        if ((2 * cp + 1 >= tc) == add) x[2 * cp + 1] = y1;
+                      }
+                    }
+                  }
+                  __syncwarp();
+                } while (tbits);
+                tmem_st32(s_tmem + c_lo, reinterpret_cast<uint32_t*>(x));
+                s_chunks |= 1u << qc;
+              }
+              if (p.skipped) {  // skipped pair-MACs of this row among the batch's pairs
+                const int nb = min(32, u - hb);
+#pragma unroll 1
+                for (int k = 0; k < nb; ++k) {
+                  const int tl = r + cen - __shfl_sync(0xffffffffu, wl, k);
+                  cnt += static_cast<unsigned long long>(tl <= 0 ? 0 : (tl < nv ? tl : nv));
+                }
+              }
             }
-          }
-          if (touched) {
-            tmem_st32(s_tmem + 64 * hc, reinterpret_cast<uint32_t*>(v));
-            tmem_st32(s_tmem + 64 * hc + 32, reinterpret_cast<uint32_t*>(v + 32));
-            stored = true;
+            tmem_st_wait();
           }
         }
+        if (SPARSE && __builtin_expect(s_chunks != 0xFu, 0)) {
+          // no S MMA on this tile: the chunks no correction wrote hold zero logits
+          uint32_t zw[32];
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) zw[cc] = 0u;
+#pragma unroll 1
+          for (int qc = 0; qc < BN / 32; ++qc)
+            if (!((s_chunks >> qc) & 1u)) tmem_st32(s_tmem + 32 * qc, zw);
+          tmem_st_wait();
+        }
+        // ---- the whole row of S in registers
+        float v[BN];
+#pragma unroll
+        for (int c = 0; c < BN; c += 32) tmem_ld32(s_tmem + c, reinterpret_cast<uint32_t*>(v + c));
+        tmem_ld_wait();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->k_empty[s]);  // this warp is done with K(j)
+        if (SPARSE && j + 1 < T) {
+          // S_g(j) is done reading Q~_g and this tile's corrections are done with
+          // the stash: zero (and stash) the pairs that die at the next tile.
+          // S_g(j+1) is issued only after this warpgroup's p_full arrival below.
+          const int zn = static_cast<int>(qr_next & 0xFF);
+          if (zn > z) {
+            zero_pairs(sQg, sh->stash[g], r, z, zn);
+            fence_proxy_async_smem();
+          }
+          zst = z;
+        }
+        qr = qr_next;
+
+        // ---- mask, max, exponentials
         if (partial) {
 #pragma unroll
-          for (int cc = 0; cc < 64; ++cc)
-            if (64 * hc + cc > cmax) v[cc] = -INFINITY;
+          for (int c = 0; c < BN; ++c)
+            if (c > cmax) v[c] = -INFINITY;
         }
+        float acc[8];
 #pragma unroll
-        for (int cc = 0; cc < 64; cc += 16)
+        for (int k = 0; k < 8; ++k) acc[k] = fmax3(v[k], v[8 + k], v[16 + k]);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) acc[k] = fmax3(acc[k], v[cc + k], v[cc + 8 + k]);
-      }
-      if (stored) tmem_st_wait();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->k_empty[s]);
-      const float mx =
-          fmaxf(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], fmax3(acc[5], acc[6], acc[7]))) * scale;
+        for (int c = 24; c < BN - 8; c += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[k] = fmax3(acc[k], v[c + k], v[c + 8 + k]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = fmaxf(acc[k], v[BN - 8 + k]);
+        const float mx =
+            fmaxf(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], fmax3(acc[5], acc[6], acc[7]))) * scale;
 
-      const float mnew = fmaxf(mrun, mx);
-      // Conditional rescale: keep the stale max until the row max has grown by
-      // more than 2^8; the final 1/l uses the same reference, so this is exact.
-      bool need = false;
-      float corr = 1.f;
-      if (mrun == -INFINITY) {
-        mrun = mnew;
-      } else if (mnew > mrun + 8.f) {
-        need = true;
-        corr = ex2_approx(mrun - mnew);
+        const float mnew = fmaxf(mrun, mx);
+        // Conditional rescale: keep the stale max until the row max has grown by
+        // more than 2^8; the final 1/l uses the same reference, so this is exact.
+        bool need = false;
+        float corr = 1.f;
+        if (mrun == -INFINITY) {
+          mrun = mnew;
+        } else if (mnew > mrun + 8.f) {
+          need = true;
+          corr = ex2_approx(mrun - mnew);
+        }
+        if (__any_sync(0xffffffffu, need)) {
+          // O_g holds PV_g up to tile j-1, issued before S_g(j); S_g(j)'s commit
+          // covers every earlier MMA, so O_g is complete here.
+#pragma unroll 1
+          for (int k = 0; k < D / 32; ++k) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_off + C::COL_O + g * D + 32 * k, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+            tmem_st32(tmem + lane_off + C::COL_O + g * D + 32 * k, o);
+          }
+          if (need) {
+            lsum2 = fmul2(lsum2, pack2(corr, corr));
+            mrun = mnew;
+          }
+        }
+        const float mref = (mrun == -INFINITY) ? 0.f : mrun;
+        const uint64_t sc2 = pack2(scale, scale), nm2 = pack2(-mref, -mref);
+        uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
+        uint32_t pw[BN / 2];
+#pragma unroll
+        for (int k = 0; k < BN / 2; ++k) {
+          const uint64_t x2 = ffma2(pack2(v[2 * k], v[2 * k + 1]), sc2, nm2);
+          float p0, p1;
+          if (exp_on_fma(k)) {
+            unpack2(exp2_poly2(x2), p0, p1);
+          } else {
+            float x0, x1;
+            unpack2(x2, x0, x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          ls[k & 3] = fadd2(ls[k & 3], pack2(p0, p1));
+          pw[k] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(s_tmem, pw);
+        tmem_st32(s_tmem + 32, pw + 32);
+        lsum2 = fadd2(lsum2, fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3])));
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&sh->p_full[g]);
       }
-      if (__any_sync(0xffffffffu, need)) {
-        // O_g holds PV(g), PV(g+2), ..., PV(j-2).  PV(j-2) was issued before S(j)
-        // and S(j)'s commit covers every earlier MMA, so O_g is complete here.
+
+      // ---- epilogue: O_g / l -> bf16
+      if (ok && warp_wait(&sh->o_done[g], 0, abort, p.err, 0x304)) {
+        tc_fence_after();
+        float l0, l1;
+        unpack2(lsum2, l0, l1);
+        const float l = l0 + l1;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + q_elem;
 #pragma unroll
         for (int k = 0; k < D / 32; ++k) {
           uint32_t o[32];
           tmem_ld32(tmem + lane_off + C::COL_O + g * D + 32 * k, o);
           tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
-          tmem_st32(tmem + lane_off + C::COL_O + g * D + 32 * k, o);
-        }
-        tmem_st_wait();
-        if (need) {
-          lsum2 = fmul2(lsum2, pack2(corr, corr));
-          mrun = mnew;
-        }
-      }
-      // ---- pass 2: p = 2^(s*scale - mref) (one packed FMA per two elements, then
-      // ex2), written back as packed bf16 P over the columns already read
-      const float mref = (mrun == -INFINITY) ? 0.f : mrun;
-      const uint64_t sc2 = pack2(scale, scale), nm2 = pack2(-mref, -mref);
-      uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-      for (int hc = 0; hc < 2; ++hc) {
-        float v[64];
-        tmem_ld32(s_tmem + 64 * hc, reinterpret_cast<uint32_t*>(v));
-        tmem_ld32(s_tmem + 64 * hc + 32, reinterpret_cast<uint32_t*>(v + 32));
-        tmem_ld_wait();
-        if (partial) {
-#pragma unroll
-          for (int cc = 0; cc < 64; ++cc)
-            if (64 * hc + cc > cmax) v[cc] = -INFINITY;
-        }
-        uint32_t pw[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          float x0, x1;
-          unpack2(ffma2(pack2(v[2 * k], v[2 * k + 1]), sc2, nm2), x0, x1);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-          ls[k & 3] = fadd2(ls[k & 3], pack2(p0, p1));
-          pw[k] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(s_tmem + 32 * hc, pw);
-      }
-      lsum2 = fadd2(lsum2, fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3])));
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&sh->p_full[j & 1]);
-    }
-
-    // ---- epilogue: merge the two groups' partial results, O / l -> bf16.  Group g
-    // writes output columns [g*d/2, (g+1)*d/2) of every row.
-    if (ok) {
-      float l0, l1;
-      unpack2(lsum2, l0, l1);
-      sh->fin_m[g][r] = mrun;
-      sh->fin_l[g][r] = l0 + l1;
-      mbar_arrive(&sh->xfin);
-      if (warp_wait(&sh->xfin, 0, abort, p.err, 0x306) && warp_wait(&sh->o_done, 0, abort, p.err, 0x304)) {
-        tc_fence_after();
-        const float ma = sh->fin_m[0][r], mb = sh->fin_m[1][r];
-        const float mm = fmaxf(ma, mb);
-        const float fa = ma == -INFINITY ? 0.f : ex2_approx(ma - mm);
-        const float fb = mb == -INFINITY ? 0.f : ex2_approx(mb - mm);
-        const float l = sh->fin_l[0][r] * fa + sh->fin_l[1][r] * fb;
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        const float wa = fa * inv, wb = fb * inv;
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + q_elem + g * (D / 2);
-#pragma unroll
-        for (int k = 0; k < D / 64; ++k) {
-          const int col = g * (D / 2) + 32 * k;
-          uint32_t oa[32], ob[32];
-          tmem_ld32(tmem + lane_off + C::COL_O + col, oa);
-          tmem_ld32(tmem + lane_off + C::COL_O + D + col, ob);
-          tmem_ld_wait();
           uint32_t ow[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            // an accumulator that received no P.V holds stale TMEM: select, never multiply
-            const float a0 = wa > 0.f ? __uint_as_float(oa[2 * e]) * wa : 0.f;
-            const float a1 = wa > 0.f ? __uint_as_float(oa[2 * e + 1]) * wa : 0.f;
-            const float b0 = wb > 0.f ? __uint_as_float(ob[2 * e]) * wb : 0.f;
-            const float b1 = wb > 0.f ? __uint_as_float(ob[2 * e + 1]) * wb : 0.f;
-            ow[e] = pack_bf16x2(a0 + b0, a1 + b1);
-          }
+          for (int e = 0; e < 16; ++e)
+            ow[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
           if (row_ok) {
             uint4* dst = reinterpret_cast<uint4*>(orow + 32 * k);
 #pragma unroll
@@ -556,11 +716,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-    }
-    if (SPARSE && p.skipped) {
+      if (SPARSE && p.skipped) {
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-      if (lane == 0 && cnt) atomicAdd(p.skipped, cnt);
+        for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+        if (lane == 0 && cnt) atomicAdd(p.skipped, cnt);
+      }
     }
   }
 
@@ -584,11 +744,19 @@ static cudaError_t launch_tc(const PrefillParams& p, const CUtensorMap& tq, cons
   if (e != cudaSuccess) return e;
   static unsigned long long configured = 0;  // one bit per device
   if (dev < 64 && !(configured & (1ull << dev))) {
+    // The register reallocation inside the kernel needs exactly the launch
+    // allocation it was written for; anything else could leave setmaxnreg.inc
+    // waiting, so refuse to launch.
+    cudaFuncAttributes attr{};
+    e = cudaFuncGetAttributes(&attr, kern);
+    if (e != cudaSuccess) return e;
+    if (attr.numRegs != kRegsLaunch) return cudaErrorInvalidKernelImage;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     configured |= 1ull << dev;
   }
-  const long long ctas = static_cast<long long>((p.q_len + BM - 1) / BM) * p.hq * p.batch;
+  const long long nqt = (p.q_len + BM - 1) / BM;
+  const long long ctas = (nqt + NQ - 1) / NQ * p.hq * p.batch;
   if (ctas == 0) return cudaSuccess;
   kern<<<static_cast<unsigned>(ctas), kThreads, bytes, s>>>(tq, tk, tv, p);
   return cudaGetLastError();
