@@ -124,6 +124,26 @@ atf_status kv_tensor_map(CUtensorMap* map, const void* base, int batch, int kv_l
   return ATF_OK;
 }
 
+// Chunk-major rotated key cache [batch][kv_heads][d/16][n_cache][16] bf16 as a
+// 5-D tensor (16 elements, token, chunk, head, batch); one box = 16 elements x
+// 128 tokens of one chunk (32-byte rows, 32-byte swizzle); tokens past n_cache
+// read as zero.
+atf_status kc_tensor_map(CUtensorMap* map, const void* base, int batch, int hkv, int d, long long n_cache) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(ATF_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+  const cuuint64_t nc = static_cast<cuuint64_t>(d / 16);
+  const cuuint64_t n = static_cast<cuuint64_t>(n_cache);
+  cuuint64_t dims[5] = {16, n, nc, static_cast<cuuint64_t>(hkv), static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[4] = {32, n * 32, nc * n * 32, static_cast<cuuint64_t>(hkv) * nc * n * 32};
+  cuuint32_t box[5] = {16, 128, 1, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ATF_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return ATF_OK;
+}
+
 // Self-test kernel: one warp waits on a barrier nobody completes, gives up after
 // `limit` cycles, records the expiry in the device error word.
 __global__ void timeout_selftest_kernel(long long limit, unsigned int* err) {
@@ -368,7 +388,10 @@ atf_status atf_decode(const void* q, const void* k_chunked, const void* v, void*
     p.v = static_cast<const char*>(v) + static_cast<size_t>(b0) * n_cache * kv_heads * d * esz;
     p.out = static_cast<char*>(out) + static_cast<size_t>(b0) * heads * d * esz;
     p.partials = static_cast<float*>(workspace) + static_cast<size_t>(b0) * heads * ns * (d + 2);
-    cudaError_t e = launch_decode(p, s);
+    CUtensorMap tv, tk;
+    if (atf_status st = kv_tensor_map(&tv, p.v, nb, static_cast<int>(n_cache), kv_heads, d)) return st;
+    if (atf_status st = kc_tensor_map(&tk, p.kc, nb, kv_heads, d, n_cache)) return st;
+    cudaError_t e = launch_decode(p, tv, tk, s);
     if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
   }
   return ATF_OK;

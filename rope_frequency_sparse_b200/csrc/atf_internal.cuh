@@ -61,7 +61,8 @@ cudaError_t launch_rope(const RopeParams& p, cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillParams& p, cudaStream_t s);
 cudaError_t launch_prefill_tc(const PrefillParams& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                               const CUtensorMap& tm_v, bool dense, cudaStream_t s);
-cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tm_v, const CUtensorMap& tm_k,
+                          cudaStream_t s);
 
 // Records a printf-style message as this thread's atf_last_error() and returns st.
 atf_status report_error(atf_status st, const char* fmt, ...);

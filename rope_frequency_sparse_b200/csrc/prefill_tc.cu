@@ -164,14 +164,6 @@ __device__ __forceinline__ void zero_pairs(uint8_t* tile, uint32_t (*stash)[BM],
   }
 }
 
-// Warp-collective bounded wait: every lane observes the barrier itself (acquire),
-// and the warp leaves together, so .sync.aligned tcgen05 ops never see a split warp.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned int* err,
-                                          unsigned int code) {
-  const bool ok = mbar_wait(bar, parity, abort, err, code);
-  return __all_sync(0xffffffffu, ok);
-}
-
 // Bounded wait that ignores the abort flag (used only while draining).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();

@@ -38,7 +38,8 @@ def test_noalloc_decode_matches_workspace_decode_twice():
 
 def test_noalloc_rejects_calls_beyond_its_fixed_scratch():
     cap = atf.atf_decode_noalloc_scratch_bytes()
-    B, Hq, Hkv, d = 200, 64, 8, 128
+    # one partial per (sequence, query head, split): 400 x 64 x 130 floats > 8 MiB
+    B, Hq, Hkv, d = 400, 64, 8, 128
     assert atf.atf_decode_workspace_bytes(B, Hq, Hkv, 1 << 20, d) > cap
     fake = 1 << 20  # never dereferenced: the call is rejected before any work
     with pytest.raises(atf.AtfError) as e:
