@@ -459,6 +459,35 @@ def run_extra(args, device, stream, flush_buf, peaks):
     return out
 
 
+def run_decode_profile(args):
+    """Only the decode step (alpha = 1) with a shortened cache, for ncu captures:
+    the decode_1m shapes with KEYS cached keys per sequence, W + K launches."""
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    w5 = synth.WORKLOADS["decode_1m"]
+    N = args.profile_decode
+    g = torch.Generator(device=device)
+    g.manual_seed(synth.DEFAULT_SEED)
+    kc = torch.randn((w5.batch, w5.kv_heads, w5.d // 16, N, 16), generator=g, device=device).to(torch.bfloat16)
+    v5 = torch.randn((w5.batch, N, w5.kv_heads, w5.d), generator=g, device=device).to(torch.bfloat16)
+    q5 = torch.randn((w5.batch, w5.q_heads, w5.d), generator=g, device=device).to(torch.bfloat16)
+    o5 = torch.empty_like(q5)
+    kv_len = np.full(w5.batch, N, dtype=np.int64)
+    ws_b = atf.atf_decode_workspace_bytes(w5.batch, w5.q_heads, w5.kv_heads, N, w5.d)
+    ws5 = torch.empty(ws_b, dtype=torch.uint8, device=device)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for it in range(args.warmup + args.steps):
+        if it == args.warmup:
+            e0.record(s)
+        atf.atf_decode(q5, kc, v5, o5, w5.batch, kv_len, N, w5.q_heads, w5.kv_heads, w5.d, w5.theta, 1.0, ws5,
+                       ws_b, None, s)
+    e1.record(s)
+    atf.atf_check(s)
+    print(json.dumps({"profile": "decode", "keys": N, "batch": w5.batch, "launches": args.warmup + args.steps,
+                      "ms_per_step": e0.elapsed_time(e1) / max(args.steps, 1)}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -467,8 +496,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="only the headline workload")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--profile-decode", type=int, metavar="KEYS", default=0,
+                    help="run only the decode step with KEYS cached keys per sequence (for ncu captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.profile_decode:
+        run_decode_profile(args)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
