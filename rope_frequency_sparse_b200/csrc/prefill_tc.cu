@@ -39,9 +39,10 @@
 // touched.  The per-tile pair ranges are tabulated in shared memory at the start.
 //
 // Exponentials.  The SFU evaluates 16 ex2 per clock per SM, as many as the
-// tensor core needs cycles for a 128x128 tile's two MMAs, so 3 of every 8 column
-// pairs evaluate 2^x on the FMA pipe instead: x = j + f with j = round(x) and
-// f in [-1/2, 1/2], 2^f by a cubic, j added to the exponent field.
+// tensor core needs cycles for a 128x128 tile's two MMAs.  A share of the column
+// pairs can evaluate 2^x on the FMA pipe instead (x = j + f with j = round(x) and
+// f in [-1/2, 1/2], 2^f by a cubic, j added to the exponent field); the share is a
+// compile-time mask, off by default (see ATF_EXP_FMA_MASK).
 #include <cuda_bf16.h>
 
 #include "atf_internal.cuh"
@@ -56,7 +57,7 @@ constexpr int NQ = 2;          // Q tiles per CTA
 constexpr int BN = 128;        // keys per KV tile
 constexpr int kThreads = 384;  // 12 warps = 3 warpgroups
 constexpr int kRegsLaunch = 168;   // registers per thread at launch (checked by the launcher)
-constexpr int kRegsCtl = 72;       // warpgroup 0 after reallocation
+constexpr int kRegsCtl = 64;       // warpgroup 0 after reallocation
 constexpr int kRegsSoftmax = 216;  // softmax warpgroups after reallocation
 static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split exceeds the launch");
 constexpr uint32_t kTmemCols = 512;
@@ -85,7 +86,7 @@ struct Cfg {
 };
 
 struct Shared {
-  uint64_t q_full[NQ], q_ready[NQ], s_full[NQ], p_full[NQ], o_done[NQ];
+  uint64_t q_full[NQ], q_ready[NQ], s_full[NQ], p_half[NQ], p_full[NQ], o_done[NQ];
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint64_t drain;
   uint32_t tmem_base;
@@ -190,10 +191,14 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
                __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
 }
 
-// column pairs k (columns 2k, 2k+1) whose exponentials use the FMA pipe
-__host__ __device__ constexpr bool exp_on_fma(int k) {
-  return (k & 7) == 1 || (k & 7) == 4 || (k & 7) == 6;
-}
+// column pairs k (columns 2k, 2k+1) whose exponentials use the FMA pipe: bit k % 8.
+// Off by default: measured on B200, this kernel is bound by its softmax -> MMA
+// dependency chain with the SFU about half busy, and every share moved to the FMA
+// pipe made both the dense and the windowed kernel slower (3/8: +7 %, 1/2: +13 %).
+#ifndef ATF_EXP_FMA_MASK
+#define ATF_EXP_FMA_MASK 0x00
+#endif
+__host__ __device__ constexpr bool exp_on_fma(int k) { return (ATF_EXP_FMA_MASK >> (k & 7)) & 1; }
 
 }  // namespace
 
@@ -242,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh->q_full[g], 1);
       mbar_init(&sh->q_ready[g], 128);
       mbar_init(&sh->s_full[g], 1);
+      mbar_init(&sh->p_half[g], 128);
       mbar_init(&sh->p_full[g], 128);
       mbar_init(&sh->o_done[g], 1);
     }
@@ -363,19 +369,27 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!(ok = warp_wait(&sh->v_full[sv], (j / NSV) & 1, abort, p.err, 0x205))) break;
               v_seen = true;
             }
-            if (!(ok = warp_wait(&sh->p_full[g], (j - jstart(g)) & 1, abort, p.err, 0x204))) break;
-            tc_fence_after();
             const uint32_t p_tmem = tmem + C::COL_S + g * BN;  // P_g(j), packed bf16 over S_g(j)
             const uint32_t o_tmem = tmem + C::COL_O + g * D;
             const uint64_t bv = dv0 + sv * kTileStep;
             const bool first = j == jstart(g);
-            if (elect_one()) {
+            // P arrives in two halves (keys 0..63, then 64..127): the first half's
+            // P.V runs while the softmax still computes the second
 #pragma unroll
-              for (int kk = 0; kk < BN / 16; ++kk)
-                mma_ts(o_tmem, p_tmem + 8 * kk, bv + ((kk * 2048) >> 4), idesc_pv, (!first || kk > 0) ? 1u : 0u);
-              if (j == T - 1) mma_commit(&sh->o_done[g]);
+            for (int half = 0; half < 2; ++half) {
+              if (!(ok = warp_wait(half ? &sh->p_full[g] : &sh->p_half[g], (j - jstart(g)) & 1, abort, p.err,
+                                   0x204 + half)))
+                break;
+              tc_fence_after();
+              if (elect_one()) {
+#pragma unroll
+                for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
+                  mma_ts(o_tmem, p_tmem + 8 * kk, bv + ((kk * 2048) >> 4), idesc_pv, (!first || kk > 0) ? 1u : 0u);
+                if (half && j == T - 1) mma_commit(&sh->o_done[g]);
+              }
+              __syncwarp();
             }
-            __syncwarp();
+            if (!ok) break;
           }
           // S_g(j+1) overwrites P_g(j); PV_g(j) was issued first and tcgen05.mma
           // operations of one thread execute in issue order.
@@ -445,12 +459,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int u = static_cast<int>((qr >> 16) & 0xFF);
         // the next tile's ranges, computed while S is still on its way
         const uint32_t qr_next = (SPARSE && j + 1 < T) ? ww.quarter_ranges(center + BN, quarter) : 0u;
-        if (!(ok = warp_wait(&sh->s_full[g], (j - j0) & 1, abort, p.err, 0x303))) break;
-        tc_fence_after();
         // valid columns of this row form the prefix [0, cmax]
         int cmax = -1;
         if (row_ok) cmax = static_cast<int>(min(static_cast<long long>(BN - 1), min(m, kv_last) - n0));
         const bool partial = __any_sync(0xffffffffu, cmax < BN - 1);
+        if (!(ok = warp_wait(&sh->s_full[g], (j - j0) & 1, abort, p.err, 0x303))) break;
+        tc_fence_after();
         // no S MMA when every pair is zeroed in every row
         const bool has_mma = !SPARSE || (ww.below(center + kZeroOffset) >> 3) < C::NCH;
         uint32_t s_chunks = has_mma ? 0xFu : 0u;  // 32-column chunks of S held in TMEM
@@ -662,6 +676,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pw[BN / 2];
 #pragma unroll
         for (int k = 0; k < BN / 2; ++k) {
+          if (k == BN / 4) {  // first half of P (keys 0..63) is complete: hand it over
+            tmem_st32(s_tmem, pw);
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&sh->p_half[g]);
+          }
           const uint64_t x2 = ffma2(pack2(v[2 * k], v[2 * k + 1]), sc2, nm2);
           float p0, p1;
           if (exp_on_fma(k)) {
@@ -675,7 +695,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           ls[k & 3] = fadd2(ls[k & 3], pack2(p0, p1));
           pw[k] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(s_tmem, pw);
         tmem_st32(s_tmem + 32, pw + 32);
         lsum2 = fadd2(lsum2, fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3])));
         tmem_st_wait();
