@@ -32,6 +32,8 @@ _lib = None
 
 F32 = 1
 BF16 = 0
+INTERLEAVED = 0   # frequency pair i = dims (2i, 2i+1), as the method's formula is written
+ROTATE_HALF = 1   # pair i = dims (i, i + d/2), NeoX-style checkpoints
 
 
 def build(force: bool = False) -> str:
@@ -54,16 +56,16 @@ def _load():
         lib.oracle_windows.argtypes = [ctypes.c_int, ctypes.c_double, ctypes.c_double, c_p, c_p]
         lib.oracle_windows.restype = None
         lib.oracle_rope.argtypes = [c_p, ctypes.c_int, c_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                    ctypes.c_int, ctypes.c_longlong, ctypes.c_double]
+                                    ctypes.c_int, ctypes.c_longlong, ctypes.c_double, ctypes.c_int]
         lib.oracle_rope.restype = None
         lib.oracle_prefill.argtypes = [c_p, c_p, c_p, ctypes.c_int, c_p, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_int, ctypes.c_longlong, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_int, ctypes.c_double, ctypes.c_double, c_p, ctypes.c_int,
-                                       ctypes.c_int]
+                                       ctypes.c_int, ctypes.c_int]
         lib.oracle_prefill.restype = ctypes.c_ulonglong
         lib.oracle_decode.argtypes = [c_p, c_p, c_p, ctypes.c_int, c_p, ctypes.c_int, ctypes.c_longlong,
                                       c_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
-                                      ctypes.c_double, ctypes.c_int]
+                                      ctypes.c_double, ctypes.c_int, ctypes.c_int]
         lib.oracle_decode.restype = ctypes.c_ulonglong
         _lib = lib
     return _lib
@@ -106,16 +108,17 @@ def windows(d: int, theta: float, alpha: float):
     return W, om
 
 
-def rope(x, theta: float, pos0: int = 0) -> np.ndarray:
-    """RoPE of x[batch][seq][heads][d] at positions pos0 + t, in fp64."""
+def rope(x, theta: float, pos0: int = 0, pairing: int = INTERLEAVED) -> np.ndarray:
+    """RoPE of x[batch][seq][heads][d] at positions pos0 + t, in fp64 (same layout)."""
     a, code = _as_raw(x)
     B, S, H, d = a.shape
     y = np.zeros((B, S, H, d), dtype=np.float64)
-    _load().oracle_rope(_ptr(a), code, _ptr(y), B, S, H, d, int(pos0), float(theta))
+    _load().oracle_rope(_ptr(a), code, _ptr(y), B, S, H, d, int(pos0), float(theta), int(pairing))
     return y
 
 
-def prefill(q, k, v, theta: float, alpha: float, q_offset: int = 0, rows=None, nthreads: int = 0):
+def prefill(q, k, v, theta: float, alpha: float, q_offset: int = 0, rows=None, nthreads: int = 0,
+            pairing: int = INTERLEAVED):
     """Causal windowed attention.  q [B][q_len][Hq][d], k/v [B][kv_len][Hkv][d].
 
     Returns (out fp64 [B][q_len][Hq][d], skipped pair count).  With ``rows``
@@ -136,11 +139,11 @@ def prefill(q, k, v, theta: float, alpha: float, q_offset: int = 0, rows=None, n
         rp, nr = _ptr(r), int(r.size)
     skipped = _load().oracle_prefill(_ptr(qa), _ptr(ka), _ptr(va), code, _ptr(out), B, q_len, kv_len,
                                      int(q_offset), Hq, Hkv, d, float(theta), float(alpha), rp, nr,
-                                     int(nthreads))
+                                     int(nthreads), int(pairing))
     return out, int(skipped)
 
 
-def decode(q, k_rot, v, kv_len, theta: float, alpha: float, nthreads: int = 0):
+def decode(q, k_rot, v, kv_len, theta: float, alpha: float, nthreads: int = 0, pairing: int = INTERLEAVED):
     """One query per sequence at position kv_len[b]-1 against an already rotated
     key cache.  q [B][Hq][d] (unrotated), k_rot/v [B][n_cache][Hkv][d].
 
@@ -156,5 +159,6 @@ def decode(q, k_rot, v, kv_len, theta: float, alpha: float, nthreads: int = 0):
     assert (kl >= 1).all() and (kl <= n_cache).all()
     out = np.zeros((B, Hq, d), dtype=np.float64)
     skipped = _load().oracle_decode(_ptr(qa), _ptr(ka), _ptr(va), code, _ptr(out), B, int(n_cache),
-                                    _ptr(kl), Hq, Hkv, d, float(theta), float(alpha), int(nthreads))
+                                    _ptr(kl), Hq, Hkv, d, float(theta), float(alpha), int(nthreads),
+                                    int(pairing))
     return out, int(skipped)

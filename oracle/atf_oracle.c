@@ -22,9 +22,14 @@
  *   s(m,n)  = (1/sqrt d) * sum_{i : m-n <= W_i} (q~_{2i} k~_{2i} + q~_{2i+1} k~_{2i+1})
  *   an empty sum gives the logit 0 (kept in the softmax, not masked);
  *   out_m   = sum_{n<=m} softmax_n(s(m,.)) v_n.
- * q~, k~ are q, k rotated by RoPE at their absolute positions, pairs (2i,2i+1):
- *   x~_{2i}   = x_{2i} cos(p omega_i) - x_{2i+1} sin(p omega_i)
- *   x~_{2i+1} = x_{2i} sin(p omega_i) + x_{2i+1} cos(p omega_i)
+ * q~, k~ are q, k rotated by RoPE at their absolute positions.  Pair i is the
+ * two dimensions (a_i, b_i): (2i, 2i+1) in the interleaved convention the
+ * method's formula is written in, (i, i + d/2) in the rotate-half convention
+ * (the one of NeoX-style checkpoints such as the Qwen2.5 family the pages
+ * measure on), `pairing` 0 and 1 below:
+ *   x~_{a_i} = x_{a_i} cos(p omega_i) - x_{b_i} sin(p omega_i)
+ *   x~_{b_i} = x_{a_i} sin(p omega_i) + x_{b_i} cos(p omega_i)
+ * and the pair product in the logit is q~_{a_i} k~_{a_i} + q~_{b_i} k~_{b_i}.
  * GQA: query head h reads key/value head floor(h / (Hq/Hkv)).
  * alpha = +inf gives W_i = INT64_MAX (plain causal RoPE attention).
  *
@@ -65,19 +70,24 @@ void oracle_windows(int d, double theta, double alpha, long long *W, double *ome
     }
 }
 
+/* The two dimensions of frequency pair i. */
+static int pair_a(int i, int d, int pairing) { return pairing ? i : 2 * i; }
+static int pair_b(int i, int d, int pairing) { return pairing ? i + d / 2 : 2 * i + 1; }
+
 /* RoPE of one head vector x (length d) at position p, into y. */
-static void rope_vec(const double *x, double *y, long long p, const double *omega, int d) {
+static void rope_vec(const double *x, double *y, long long p, const double *omega, int d, int pairing) {
     for (int i = 0; i < d / 2; ++i) {
+        const int a = pair_a(i, d, pairing), b = pair_b(i, d, pairing);
         double phi = (double)p * omega[i];
         double c = cos(phi), s = sin(phi);
-        y[2 * i] = x[2 * i] * c - x[2 * i + 1] * s;
-        y[2 * i + 1] = x[2 * i] * s + x[2 * i + 1] * c;
+        y[a] = x[a] * c - x[b] * s;
+        y[b] = x[a] * s + x[b] * c;
     }
 }
 
 /* Rotate x[b][t][h][d] (dtype) at positions pos0 + t; y is fp64, same layout. */
 void oracle_rope(const void *x, int dtype, double *y, int batch, int seq, int heads, int d,
-                 long long pos0, double theta) {
+                 long long pos0, double theta, int pairing) {
     double *omega = malloc(sizeof(double) * (size_t)(d / 2));
     long long *W = malloc(sizeof(long long) * (size_t)(d / 2));
     double *xv = malloc(sizeof(double) * (size_t)d);
@@ -87,7 +97,7 @@ void oracle_rope(const void *x, int dtype, double *y, int batch, int seq, int he
             for (int h = 0; h < heads; ++h) {
                 long long base = (((long long)b * seq + t) * heads + h) * d;
                 for (int e = 0; e < d; ++e) xv[e] = widen(x, base + e, dtype);
-                rope_vec(xv, y + base, pos0 + t, omega, d);
+                rope_vec(xv, y + base, pos0 + t, omega, d, pairing);
             }
     free(omega);
     free(W);
@@ -105,6 +115,7 @@ typedef struct {
     long long q_offset;
     const long long *W;
     const double *omega;
+    int pairing;     /* 0: pairs (2i, 2i+1); 1: pairs (i, i + d/2) */
     const int *rows; /* NULL: all t */
     int n_rows;
     const double *k64;  /* keys rotated once up front (fp64), or NULL: k is already rotated */
@@ -120,7 +131,7 @@ static void one_row(job_t *J, int b, int h, int t, double *qt, double *kt, doubl
     double *qraw = malloc(sizeof(double) * (size_t)d);
     long long qbase = (((long long)b * J->q_len + t) * J->Hq + h) * d;
     for (int e = 0; e < d; ++e) qraw[e] = widen(J->q, qbase + e, J->dtype);
-    rope_vec(qraw, qt, m, J->omega, d);
+    rope_vec(qraw, qt, m, J->omega, d, J->pairing);
     free(qraw);
 
     long long nmax = m;
@@ -136,8 +147,9 @@ static void one_row(job_t *J, int b, int h, int t, double *qt, double *kt, doubl
         long long delta = m - n;
         double acc = 0.0;
         for (int i = 0; i < d / 2; ++i) {
+            const int a = pair_a(i, d, J->pairing), bb = pair_b(i, d, J->pairing);
             if (delta <= J->W[i])
-                acc += qt[2 * i] * kt[2 * i] + qt[2 * i + 1] * kt[2 * i + 1];
+                acc += qt[a] * kt[a] + qt[bb] * kt[bb];
             else
                 *skipped += 1;
         }
@@ -209,7 +221,7 @@ static unsigned long long run_jobs(job_t *J, int nthreads) {
 unsigned long long oracle_prefill(const void *q, const void *k, const void *v, int dtype, double *out,
                                   int batch, int q_len, int kv_len, long long q_offset, int Hq, int Hkv,
                                   int d, double theta, double alpha, const int *rows, int n_rows,
-                                  int nthreads) {
+                                  int nthreads, int pairing) {
     long long *W = malloc(sizeof(long long) * (size_t)(d / 2));
     double *omega = malloc(sizeof(double) * (size_t)(d / 2));
     oracle_windows(d, theta, alpha, W, omega);
@@ -218,9 +230,10 @@ unsigned long long oracle_prefill(const void *q, const void *k, const void *v, i
     J.q = q; J.k = k; J.v = v; J.dtype = dtype; J.out = out;
     J.batch = batch; J.q_len = q_len; J.kv_len = kv_len; J.Hq = Hq; J.Hkv = Hkv; J.d = d;
     J.q_offset = q_offset; J.W = W; J.omega = omega; J.rows = rows; J.n_rows = n_rows;
+    J.pairing = pairing;
     /* keys are rotated once, at their absolute positions 0..kv_len-1 */
     double *k64 = malloc(sizeof(double) * (size_t)batch * (size_t)kv_len * (size_t)Hkv * (size_t)d);
-    oracle_rope(k, dtype, k64, batch, kv_len, Hkv, d, 0, theta);
+    oracle_rope(k, dtype, k64, batch, kv_len, Hkv, d, 0, theta, pairing);
     J.k64 = k64;
     unsigned long long s = run_jobs(&J, nthreads);
     free(k64);
@@ -231,13 +244,13 @@ unsigned long long oracle_prefill(const void *q, const void *k, const void *v, i
 
 /*
  * Decode oracle: one new query per sequence.  q: raw (unrotated) [batch][Hq][d];
- * k_rot: keys ALREADY rotated, [batch][n_cache][Hkv][d]; v: [batch][n_cache][Hkv][d];
+ * k_rot: keys ALREADY rotated (same pairing), [batch][n_cache][Hkv][d]; v: [batch][n_cache][Hkv][d];
  * kv_len[b] <= n_cache keys are live; the query sits at position kv_len[b]-1.
  * out: fp64 [batch][Hq][d].  Returns the skipped pair count.
  */
 unsigned long long oracle_decode(const void *q, const void *k_rot, const void *v, int dtype, double *out,
                                  int batch, long long n_cache, const long long *kv_len, int Hq, int Hkv,
-                                 int d, double theta, double alpha, int nthreads) {
+                                 int d, double theta, double alpha, int nthreads, int pairing) {
     long long *W = malloc(sizeof(long long) * (size_t)(d / 2));
     double *omega = malloc(sizeof(double) * (size_t)(d / 2));
     oracle_windows(d, theta, alpha, W, omega);
@@ -255,6 +268,7 @@ unsigned long long oracle_decode(const void *q, const void *k_rot, const void *v
         J.batch = 1; J.q_len = 1; J.kv_len = (int)kv_len[b]; J.Hq = Hq; J.Hkv = Hkv; J.d = d;
         J.q_offset = kv_len[b] - 1; J.W = W; J.omega = omega; J.rows = NULL; J.n_rows = 0;
         J.k64 = NULL;
+        J.pairing = pairing;
         total += run_jobs(&J, nthreads);
     }
     free(W);

@@ -290,3 +290,87 @@ def test_sampled_rows_match_full():
     part, _ = oracle.prefill(q, k, v, 1e4, 1.0, rows=rows)
     assert np.abs(part[:, rows] - full[:, rows]).max() == 0.0
     assert np.isnan(part[:, 1]).all()
+
+
+# --------------------------------------------------------------------------- rotate-half pairing
+
+def _half_to_interleaved(x):
+    """Reorder the last axis so that rotate-half pair i = dims (i, i + d/2) lands on
+    dims (2i, 2i+1)."""
+    d = x.shape[-1]
+    perm = np.empty(d, dtype=np.int64)
+    perm[0::2] = np.arange(d // 2)
+    perm[1::2] = np.arange(d // 2) + d // 2
+    return x[..., perm]
+
+
+def _rotate_half_complex(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
+    """Rotate-half RoPE as complex multiplication: pair i is x_i + j x_{i+d/2}."""
+    d = x.shape[-1]
+    omega = np.exp(-(2.0 * np.arange(d // 2) / d) * np.log(theta))
+    z = x[..., : d // 2] + 1j * x[..., d // 2:]
+    z = z * np.exp(1j * pos[None, :, None, None] * omega[None, None, None, :])
+    return np.concatenate([z.real, z.imag], axis=-1)
+
+
+def test_rotate_half_rope_unit_vectors():
+    """A unit vector in dim i (< d/2) at position p rotates to cos p omega_i in dim i
+    and sin p omega_i in dim i + d/2; a unit vector in dim i + d/2 to -sin, cos."""
+    d, theta = 8, 100.0
+    eye = np.eye(d, dtype=np.float32)
+    for i in range(d // 2):
+        om = theta ** (-2 * i / d)
+        for p in (0, 1, 7, 2**20 - 1):
+            a = oracle.rope(eye[i].reshape(1, 1, 1, d), theta, pos0=p, pairing=oracle.ROTATE_HALF)[0, 0, 0]
+            b = oracle.rope(eye[i + d // 2].reshape(1, 1, 1, d), theta, pos0=p, pairing=oracle.ROTATE_HALF)[0, 0, 0]
+            assert abs(a[i] - math.cos(p * om)) < 1e-12 and abs(a[i + d // 2] - math.sin(p * om)) < 1e-12
+            assert abs(b[i] + math.sin(p * om)) < 1e-12 and abs(b[i + d // 2] - math.cos(p * om)) < 1e-12
+            assert np.abs(np.delete(a, [i, i + d // 2])).max() == 0
+            assert np.abs(np.delete(b, [i, i + d // 2])).max() == 0
+
+
+def test_rotate_half_rope_matches_complex_form():
+    q, _, _ = synth.random_prefill(2, 21, 21, 3, 3, 16, torch.float32, seed=13)
+    y = oracle.rope(q, 1e4, pos0=5, pairing=oracle.ROTATE_HALF)
+    want = _rotate_half_complex(q.double().numpy(), np.arange(5, 26, dtype=np.float64), 1e4)
+    assert np.abs(y - want).max() < 1e-12
+
+
+@pytest.mark.parametrize("alpha", [0.5, 1.0, math.inf])
+def test_rotate_half_equals_interleaved_on_reordered_dims(alpha):
+    """Pair i of the rotate-half convention is pair i of the interleaved one once
+    dims (i, i+d/2) are moved to (2i, 2i+1) in q and k (v untouched): the same
+    windows, logits, outputs and skipped pairs."""
+    B, S, Hq, Hkv, d, theta = 1, 70, 4, 2, 16, 100.0
+    q, k, v = synth.random_prefill(B, S, S, Hq, Hkv, d, torch.float32, seed=17)
+    out_h, sk_h = oracle.prefill(q, k, v, theta, alpha, pairing=oracle.ROTATE_HALF)
+    qi = torch.from_numpy(np.ascontiguousarray(_half_to_interleaved(q.numpy())))
+    ki = torch.from_numpy(np.ascontiguousarray(_half_to_interleaved(k.numpy())))
+    out_i, sk_i = oracle.prefill(qi, ki, v, theta, alpha, pairing=oracle.INTERLEAVED)
+    assert sk_h == sk_i
+    assert np.abs(out_h - out_i).max() < 1e-12
+    W, _ = oracle.windows(d, theta, alpha)
+    assert sk_h == Hq * sum(_tri(S - 1 - int(w)) for w in W)
+
+
+def test_rotate_half_dense_case_equals_sdpa():
+    B, S, Hq, Hkv, d, theta = 2, 29, 4, 2, 16, 100.0
+    q, k, v = synth.random_prefill(B, S, S, Hq, Hkv, d, torch.float32, seed=19)
+    out, skipped = oracle.prefill(q, k, v, theta, math.inf, pairing=oracle.ROTATE_HALF)
+    assert skipped == 0
+    pos = np.arange(S, dtype=np.float64)
+    qr = torch.from_numpy(_rotate_half_complex(q.double().numpy(), pos, theta))
+    kr = torch.from_numpy(_rotate_half_complex(k.double().numpy(), pos, theta))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        qr.transpose(1, 2), kr.transpose(1, 2), v.double().transpose(1, 2), is_causal=True, enable_gqa=True)
+    assert np.abs(out - ref.transpose(1, 2).numpy()).max() < 1e-12
+
+
+def test_rotate_half_decode_equals_last_prefill_row():
+    B, S, Hq, Hkv, d, theta = 1, 45, 4, 2, 16, 100.0
+    q, k, v = synth.random_prefill(B, S, S, Hq, Hkv, d, torch.float32, seed=23)
+    out_p, _ = oracle.prefill(q, k, v, theta, 1.0, pairing=oracle.ROTATE_HALF)
+    k_rot = torch.from_numpy(oracle.rope(k, theta, pairing=oracle.ROTATE_HALF).astype(np.float32))
+    out_d, _ = oracle.decode(q[:, -1], k_rot, v, [S], theta, 1.0, pairing=oracle.ROTATE_HALF)
+    # the decode path reads k rotated once to fp32; compare at fp32 rounding of k~
+    assert np.abs(out_d - out_p[:, -1]).max() < 1e-5
