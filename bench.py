@@ -171,16 +171,18 @@ class PrefillStep:
         self.k_rot = self.ws[off: off + B * S * Hkv * d * 2].view(torch.bfloat16).view(B, S, Hkv, d)
         self.cnt = torch.zeros(1, dtype=torch.int64, device=device)
 
-    def run(self, alpha, stream, ev=None):
+    def run(self, alpha, stream, ev=None, pairing=0):
         """RoPE q, RoPE k, windowed prefill: 3 kernel launches.  ev = (e0, e1, e2)
-        brackets the RoPE part and the prefill kernel."""
+        brackets the RoPE part and the prefill kernel.  pairing 1 reads q, k as
+        rotate-half (NeoX-style) pairs."""
         w = self.w
         B, S, Hq, d = self.q.shape
         Hkv = self.k.shape[2]
+        mode = 2 if pairing == atf.ATF_PAIRS_ROTATE_HALF else 1
         if ev:
             ev[0].record(stream)
-        atf.atf_rope_layout(self.q, self.q_rot, None, B, S, Hq, d, 0, w.theta, 1, atf.ATF_BF16, stream)
-        atf.atf_rope_layout(self.k, self.k_rot, None, B, S, Hkv, d, 0, w.theta, 1, atf.ATF_BF16, stream)
+        atf.atf_rope_layout(self.q, self.q_rot, None, B, S, Hq, d, 0, w.theta, mode, atf.ATF_BF16, stream)
+        atf.atf_rope_layout(self.k, self.k_rot, None, B, S, Hkv, d, 0, w.theta, mode, atf.ATF_BF16, stream)
         if ev:
             ev[1].record(stream)
         atf.atf_prefill_ex(self.q_rot, self.k_rot, self.v, self.out, B, S, S, Hq, Hkv, d, 0, atf.ATF_BF16, 1,
@@ -370,9 +372,20 @@ def run_ours(args, rank, world, local_rank):
 
 
 def run_extra(args, device, stream, flush_buf, peaks):
-    """Secondary workloads: 32k pair-energy prefill, 128k chunked prefill, 1M-key decode."""
+    """Secondary workloads: the 8k step with rotate-half pairs, 32k pair-energy
+    prefill, 128k chunked prefill, 1M-key decode."""
     s = stream
     out = {}
+    # the headline 8k step with q, k read as rotate-half (NeoX-style) pairs
+    w2 = synth.WORKLOADS[HEADLINE]
+    st2 = PrefillStep(w2, synth.DEFAULT_SEED, device)
+    ev2 = time_steps(lambda ev: st2.run(1.0, s, ev, pairing=atf.ATF_PAIRS_ROTATE_HALF), 5, 3, stream, flush_buf)
+    ms2 = sum(e[0].elapsed_time(e[2]) for e in ev2) / 5
+    ms2r = sum(e[0].elapsed_time(e[1]) for e in ev2) / 5
+    eff2 = prefill_flops(w2, 1.0)[0]
+    out["layer_8k_rotate_half"] = {"tflops": eff2 / (ms2 * 1e-3) / 1e12, "ms": ms2, "rope_ms": ms2r}
+    del st2
+    torch.cuda.empty_cache()
     # 32k tokens, pair-energy-scaled q/k
     w3 = synth.WORKLOADS["layer_32k_pair_energy"]
     st3 = PrefillStep(w3, synth.DEFAULT_SEED, device)

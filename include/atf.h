@@ -50,6 +50,14 @@ typedef enum {
 
 typedef enum { ATF_BF16 = 0, ATF_FP32 = 1 } atf_dtype;
 
+/* Which dimensions form RoPE frequency pair i (i < d/2): (2i, 2i+1) as in the
+ * method's formula, or (i, i + d/2) as in rotate-half (NeoX-style) checkpoints
+ * such as the Qwen2.5 family the pages measure on.  Pair i has the same
+ * frequency theta^(-2i/d) and window W_i either way.  The attention kernels read
+ * rotated queries and keys in the interleaved order; atf_rope_layout's
+ * rotate-half modes write rotate-half pairs in that order. */
+typedef enum { ATF_PAIRS_INTERLEAVED = 0, ATF_PAIRS_ROTATE_HALF = 1 } atf_pairing;
+
 /* Window table.  Writes W_i = ceil(alpha * 2 pi / theta^(-2i/d)), i < d/2, into
  * the host array W_out (d/2 entries), evaluated in fp64.  alpha = +inf gives
  * INT64_MAX.  Host only; no GPU needed. */
@@ -63,8 +71,14 @@ atf_status atf_windows(int d, double theta, double alpha, long long* W_out);
  *   x_chunked: output [batch][heads][d/16][seq][16] (bf16 only), may be NULL:
  *              the pair-chunk-major key layout read by atf_decode (chunk c holds
  *              pairs 8c..8c+7 of every token contiguously).
- *   rotate:    1 = apply RoPE, 0 = copy / re-layout only (for caches already
- *              rotated). */
+ *   rotate:    0 = copy / re-layout only (for caches already rotated),
+ *              1 = apply RoPE to interleaved pairs (2i, 2i+1),
+ *              2 = apply RoPE to rotate-half pairs (i, i + d/2) and write pair i
+ *                  to dims (2i, 2i+1) of x_rot / x_chunked (the order the
+ *                  attention kernels read; x and x_rot must not alias),
+ *              3 = no rotation, only that reordering (rotate-half caches that
+ *                  are already rotated).
+ *              Other values: ATF_ERR_INVALID_ARG. */
 atf_status atf_rope_layout(const void* x, void* x_rot, void* x_chunked, int batch, int seq, int heads, int d,
                            long long pos_offset, double theta, int rotate, int dtype, void* stream);
 
@@ -77,12 +91,14 @@ typedef struct {
   int batch, q_len, kv_len, heads, kv_heads, d;
   long long q_offset; /* absolute position of query row 0; kv_len >= q_offset + q_len */
   int dtype;          /* atf_dtype: ATF_BF16 -> tensor-core kernel, ATF_FP32 -> fp32 CUDA-core kernel */
-  int rotated;        /* 1: q and k are already RoPE-rotated (e.g. by atf_rope_layout) */
+  int rotated;        /* 1: q and k are already RoPE-rotated and in the kernels' interleaved
+                         pair order (e.g. by atf_rope_layout); 0: rotated here */
   double theta, alpha;
   unsigned long long* skipped_pairs; /* device, may be NULL: += number of (query head, query,
                                         key, pair) quadruples outside their window */
   void* workspace;                   /* device scratch for the rotated q, k when rotated == 0 */
   size_t workspace_bytes;            /* >= atf_prefill_workspace_bytes(...) when rotated == 0 */
+  int pairing;        /* atf_pairing of the unrotated q, k (used when rotated == 0) */
 } atf_prefill_args;
 
 /* Scratch bytes atf_prefill_ex needs for rotated copies of q and k (0 if rotated). */
@@ -102,7 +118,9 @@ atf_status atf_prefill(const void* q, const void* k, const void* v, void* out, i
                        int d, double theta, double alpha, void* stream);
 
 /* Decode: one new query per sequence against a rotated key cache.
- *   q:          [batch][heads][d] bf16, NOT rotated; rotated here at position kv_len[b]-1.
+ *   q:          [batch][heads][d] bf16, NOT rotated; rotated here at position kv_len[b]-1
+ *               with the given atf_pairing.
+ *   pairing:    atf_pairing of q (the cache is in the interleaved pair order either way).
  *   k_chunked:  [batch][kv_heads][d/16][n_cache][16] bf16, keys already rotated at
  *               their positions, pair-chunk-major (see atf_rope_layout).
  *   v:          [batch][n_cache][kv_heads][d] bf16.
@@ -117,8 +135,8 @@ atf_status atf_prefill(const void* q, const void* k, const void* v, void* out, i
  * from memory; every value row is read. */
 atf_status atf_decode(const void* q, const void* k_chunked, const void* v, void* out, int batch,
                       const long long* kv_len, long long n_cache, int heads, int kv_heads, int d, double theta,
-                      double alpha, void* workspace, size_t workspace_bytes, unsigned long long* skipped_pairs,
-                      void* stream);
+                      double alpha, int pairing, void* workspace, size_t workspace_bytes,
+                      unsigned long long* skipped_pairs, void* stream);
 
 /* Scratch bytes atf_decode needs for `batch` sequences of at most max_kv_len keys. */
 size_t atf_decode_workspace_bytes(int batch, int heads, int kv_heads, long long max_kv_len, int d);
@@ -144,7 +162,8 @@ size_t atf_decode_workspace_bytes(int batch, int heads, int kv_heads, long long 
  *     kernels overlap on the GPU (e.g. on unordered streams) race on it. */
 atf_status atf_decode_noalloc(const void* q, const void* k_chunked, const void* v, void* out, int batch,
                               const long long* kv_len, long long n_cache, int heads, int kv_heads, int d,
-                              double theta, double alpha, unsigned long long* skipped_pairs, void* stream);
+                              double theta, double alpha, int pairing, unsigned long long* skipped_pairs,
+                              void* stream);
 
 /* Size in bytes of atf_decode_noalloc's fixed device scratch array. */
 size_t atf_decode_noalloc_scratch_bytes(void);

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libatf.so")
 
 ATF_OK, ATF_ERR_INVALID_ARG, ATF_ERR_UNSUPPORTED, ATF_ERR_CUDA, ATF_ERR_TIMEOUT = range(5)
 ATF_BF16, ATF_FP32 = 0, 1
+ATF_PAIRS_INTERLEAVED, ATF_PAIRS_ROTATE_HALF = 0, 1
 STATUS_NAMES = {0: "ATF_OK", 1: "ATF_ERR_INVALID_ARG", 2: "ATF_ERR_UNSUPPORTED", 3: "ATF_ERR_CUDA",
                 4: "ATF_ERR_TIMEOUT"}
 
@@ -40,6 +41,7 @@ class PrefillArgs(ctypes.Structure):
         ("theta", ctypes.c_double), ("alpha", ctypes.c_double),
         ("skipped_pairs", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("pairing", ctypes.c_int),
     ]
 
 
@@ -62,9 +64,9 @@ def load_library(path: str = LIB_PATH):
         "atf_prefill_workspace_bytes": ([i, i, i, i, i, i, i, i], sz),
         "atf_prefill_ex": ([ctypes.POINTER(PrefillArgs), vp], i),
         "atf_prefill": ([vp, vp, vp, vp, i, i, i, i, d, d, vp], i),
-        "atf_decode": ([vp, vp, vp, vp, i, vp, ll, i, i, i, d, d, vp, sz, vp, vp], i),
+        "atf_decode": ([vp, vp, vp, vp, i, vp, ll, i, i, i, d, d, i, vp, sz, vp, vp], i),
         "atf_decode_workspace_bytes": ([i, i, i, ll, i], sz),
-        "atf_decode_noalloc": ([vp, vp, vp, vp, i, vp, ll, i, i, i, d, d, vp, vp], i),
+        "atf_decode_noalloc": ([vp, vp, vp, vp, i, vp, ll, i, i, i, d, d, i, vp, vp], i),
         "atf_decode_noalloc_scratch_bytes": ([], sz),
         "atf_check": ([vp], i),
         "atf_selftest_timeout": ([ll, vp], i),
@@ -133,10 +135,10 @@ def atf_prefill_workspace_bytes(batch, q_len, kv_len, heads, kv_heads, d, dtype,
 
 
 def atf_prefill_ex(q, k, v, out, batch, q_len, kv_len, heads, kv_heads, d, q_offset, dtype, rotated, theta, alpha,
-                   skipped_pairs=None, workspace=None, workspace_bytes=0, stream=None):
+                   skipped_pairs=None, workspace=None, workspace_bytes=0, stream=None, pairing=ATF_PAIRS_INTERLEAVED):
     a = PrefillArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(out), batch, q_len, kv_len, heads, kv_heads, d, int(q_offset),
                     int(dtype), int(rotated), float(theta), float(alpha), _ptr(skipped_pairs), _ptr(workspace),
-                    int(workspace_bytes))
+                    int(workspace_bytes), int(pairing))
     _check(load_library().atf_prefill_ex(ctypes.byref(a), _stream(stream)))
 
 
@@ -146,21 +148,22 @@ def atf_prefill(q, k, v, out, seq, heads, kv_heads, d, theta, alpha, stream=None
 
 
 def atf_decode(q, k_chunked, v, out, batch, kv_len, n_cache, heads, kv_heads, d, theta, alpha, workspace,
-               workspace_bytes, skipped_pairs=None, stream=None):
+               workspace_bytes, skipped_pairs=None, stream=None, pairing=ATF_PAIRS_INTERLEAVED):
     kl = np.ascontiguousarray(np.asarray(kv_len, dtype=np.int64).reshape(-1))
     _check(load_library().atf_decode(_ptr(q), _ptr(k_chunked), _ptr(v), _ptr(out), batch,
                                      kl.ctypes.data_as(ctypes.c_void_p), int(n_cache), heads, kv_heads, d,
-                                     float(theta), float(alpha), _ptr(workspace), int(workspace_bytes),
-                                     _ptr(skipped_pairs), _stream(stream)))
+                                     float(theta), float(alpha), int(pairing), _ptr(workspace),
+                                     int(workspace_bytes), _ptr(skipped_pairs), _stream(stream)))
 
 
 def atf_decode_noalloc(q, k_chunked, v, out, batch, kv_len, n_cache, heads, kv_heads, d, theta, alpha,
-                       skipped_pairs=None, stream=None):
+                       skipped_pairs=None, stream=None, pairing=ATF_PAIRS_INTERLEAVED):
     """atf_decode with its scratch in the library's fixed device array (no allocation)."""
     kl = np.ascontiguousarray(np.asarray(kv_len, dtype=np.int64).reshape(-1))
     _check(load_library().atf_decode_noalloc(_ptr(q), _ptr(k_chunked), _ptr(v), _ptr(out), batch,
                                              kl.ctypes.data_as(ctypes.c_void_p), int(n_cache), heads, kv_heads, d,
-                                             float(theta), float(alpha), _ptr(skipped_pairs), _stream(stream)))
+                                             float(theta), float(alpha), int(pairing), _ptr(skipped_pairs),
+                                             _stream(stream)))
 
 
 def atf_decode_noalloc_scratch_bytes() -> int:
@@ -181,18 +184,22 @@ def atf_selftest_timeout(limit_cycles: int, stream=None):
 
 # ------------------------------------------------------------------ torch conveniences (allocation only)
 
-def rope_layout(x, theta, pos_offset=0, rotated_out=True, chunked_out=False, rotate=True, stream=None):
-    """Rotate x [B][S][H][d] (torch, CUDA); returns (x_rot or None, x_chunked or None)."""
+def rope_layout(x, theta, pos_offset=0, rotated_out=True, chunked_out=False, rotate=True, stream=None,
+                pairing=ATF_PAIRS_INTERLEAVED):
+    """Rotate x [B][S][H][d] (torch, CUDA); returns (x_rot or None, x_chunked or None).
+    With rotate-half pairing the outputs hold pair i in dims (2i, 2i+1)."""
     import torch
 
     B, S, H, d = x.shape
     xr = torch.empty_like(x) if rotated_out else None
     xc = torch.empty((B, H, d // 16, S, 16), dtype=x.dtype, device=x.device) if chunked_out else None
-    atf_rope_layout(x, xr, xc, B, S, H, d, pos_offset, theta, 1 if rotate else 0, dtype_code(x), stream)
+    mode = (2 if rotate else 3) if pairing == ATF_PAIRS_ROTATE_HALF else (1 if rotate else 0)
+    atf_rope_layout(x, xr, xc, B, S, H, d, pos_offset, theta, mode, dtype_code(x), stream)
     return xr, xc
 
 
-def prefill(q, k, v, theta, alpha, q_offset=0, rotated=False, skipped=None, out=None, workspace=None, stream=None):
+def prefill(q, k, v, theta, alpha, q_offset=0, rotated=False, skipped=None, out=None, workspace=None, stream=None,
+            pairing=ATF_PAIRS_INTERLEAVED):
     """Windowed causal prefill; q [B][q_len][Hq][d], k/v [B][kv_len][Hkv][d] (torch, CUDA)."""
     import torch
 
@@ -205,11 +212,12 @@ def prefill(q, k, v, theta, alpha, q_offset=0, rotated=False, skipped=None, out=
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     atf_prefill_ex(q, k, v, out, B, q_len, kv_len, Hq, Hkv, d, q_offset, dt, int(rotated), theta, alpha,
-                   skipped, workspace, need, stream)
+                   skipped, workspace, need, stream, pairing)
     return out
 
 
-def decode(q, k_chunked, v, kv_len, theta, alpha, skipped=None, out=None, workspace=None, stream=None):
+def decode(q, k_chunked, v, kv_len, theta, alpha, skipped=None, out=None, workspace=None, stream=None,
+           pairing=ATF_PAIRS_INTERLEAVED):
     """Decode step; q [B][Hq][d], k_chunked [B][Hkv][d/16][N][16], v [B][N][Hkv][d] (torch, CUDA)."""
     import torch
 
@@ -221,7 +229,7 @@ def decode(q, k_chunked, v, kv_len, theta, alpha, skipped=None, out=None, worksp
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     if out is None:
         out = torch.empty_like(q)
-    atf_decode(q, k_chunked, v, out, B, kl, N, Hq, Hkv, d, theta, alpha, workspace, need, skipped, stream)
+    atf_decode(q, k_chunked, v, out, B, kl, N, Hq, Hkv, d, theta, alpha, workspace, need, skipped, stream, pairing)
     return out
 
 

@@ -192,6 +192,7 @@ atf_status atf_rope_layout(const void* x, void* x_rot, void* x_chunked, int batc
   if (batch < 0 || seq < 0 || heads < 1 || pos_offset < 0)
     return fail(ATF_ERR_INVALID_ARG, "rope_layout: bad sizes");
   if (dtype != ATF_BF16 && dtype != ATF_FP32) return fail(ATF_ERR_INVALID_ARG, "bad dtype %d", dtype);
+  if (rotate < 0 || rotate > 3) return fail(ATF_ERR_INVALID_ARG, "rope_layout: rotate %d", rotate);
   if (x_chunked && dtype != ATF_BF16) return fail(ATF_ERR_UNSUPPORTED, "chunk-major layout is bf16 only");
   if (static_cast<long long>(batch) * seq == 0) return ATF_OK;
   if (!x || (!x_rot && !x_chunked)) return fail(ATF_ERR_INVALID_ARG, "rope_layout: null pointer");
@@ -206,7 +207,7 @@ atf_status atf_rope_layout(const void* x, void* x_rot, void* x_chunked, int batc
   p.heads = heads;
   p.d = d;
   p.pos_offset = pos_offset;
-  p.rotate = rotate ? 1 : 0;
+  p.rotate = rotate;
   p.fp32 = dtype == ATF_FP32;
   Windows w;
   kernel_windows(d, theta, INFINITY, &w, p.omega);
@@ -230,6 +231,8 @@ atf_status atf_prefill_ex(const atf_prefill_args* a, void* stream) {
   if (a->dtype != ATF_BF16 && a->dtype != ATF_FP32) return fail(ATF_ERR_INVALID_ARG, "bad dtype %d", a->dtype);
   if (a->batch < 0 || a->q_len < 0 || a->kv_len < 0 || a->q_offset < 0 || a->heads < 1 || a->kv_heads < 1)
     return fail(ATF_ERR_INVALID_ARG, "prefill: negative or zero sizes");
+  if (a->pairing != ATF_PAIRS_INTERLEAVED && a->pairing != ATF_PAIRS_ROTATE_HALF)
+    return fail(ATF_ERR_INVALID_ARG, "prefill: pairing %d", a->pairing);
   if (a->heads % a->kv_heads) return fail(ATF_ERR_INVALID_ARG, "heads %% kv_heads != 0");
   if (static_cast<long long>(a->kv_len) < a->q_offset + a->q_len)
     return fail(ATF_ERR_INVALID_ARG, "prefill: kv_len (%d) < q_offset + q_len (%lld)", a->kv_len,
@@ -258,11 +261,12 @@ atf_status atf_prefill_ex(const atf_prefill_args* a, void* stream) {
     void* q_rot = ws;
     void* k_rot = ws + round_up(static_cast<size_t>(a->batch) * a->q_len * a->heads * a->d * esz, 256);
     // queries at positions q_offset + t, keys at positions n (every batch entry alike)
+    const int mode = a->pairing == ATF_PAIRS_ROTATE_HALF ? 2 : 1;  // rotate-half pairs end up interleaved
     atf_status st = atf_rope_layout(a->q, q_rot, nullptr, a->batch, a->q_len, a->heads, a->d, a->q_offset,
-                                    a->theta, 1, a->dtype, stream);
+                                    a->theta, mode, a->dtype, stream);
     if (st) return st;
-    st = atf_rope_layout(a->k, k_rot, nullptr, a->batch, a->kv_len, a->kv_heads, a->d, 0, a->theta, 1, a->dtype,
-                         stream);
+    st = atf_rope_layout(a->k, k_rot, nullptr, a->batch, a->kv_len, a->kv_heads, a->d, 0, a->theta, mode,
+                         a->dtype, stream);
     if (st) return st;
     q = q_rot;
     k = k_rot;
@@ -341,9 +345,11 @@ size_t atf_decode_workspace_bytes(int batch, int heads, int kv_heads, long long 
 
 atf_status atf_decode(const void* q, const void* k_chunked, const void* v, void* out, int batch,
                       const long long* kv_len, long long n_cache, int heads, int kv_heads, int d, double theta,
-                      double alpha, void* workspace, size_t workspace_bytes, unsigned long long* skipped_pairs,
-                      void* stream) {
+                      double alpha, int pairing, void* workspace, size_t workspace_bytes,
+                      unsigned long long* skipped_pairs, void* stream) {
   if (atf_status st = check_params(d, theta, alpha)) return st;
+  if (pairing != ATF_PAIRS_INTERLEAVED && pairing != ATF_PAIRS_ROTATE_HALF)
+    return fail(ATF_ERR_INVALID_ARG, "decode: pairing %d", pairing);
   if (batch < 0 || heads < 1 || kv_heads < 1 || n_cache < 1) return fail(ATF_ERR_INVALID_ARG, "decode: bad sizes");
   if (heads % kv_heads) return fail(ATF_ERR_INVALID_ARG, "heads %% kv_heads != 0");
   if (heads / kv_heads > 8) return fail(ATF_ERR_UNSUPPORTED, "decode: at most 8 query heads per kv head");
@@ -375,6 +381,7 @@ atf_status atf_decode(const void* q, const void* k_chunked, const void* v, void*
   p.hkv = kv_heads;
   p.d = d;
   p.n_split = ns;
+  p.pairing = pairing;
   p.n_cache = n_cache;
   p.skipped = skipped_pairs;
   p.err = err;

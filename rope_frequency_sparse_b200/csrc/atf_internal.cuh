@@ -24,7 +24,7 @@ struct RopeParams {
   void* x_chunked;  // nullable, bf16 only: [B][H][d/16][S][16]
   int batch, seq, heads, d;
   long long pos_offset;
-  int rotate;  // 0: layout copy only
+  int rotate;  // 0: copy, 1: RoPE, 2: rotate-half RoPE, 3: rotate-half copy (2, 3 write pairs interleaved)
   int fp32;    // 1: fp32 elements, 0: bf16
   double omega[kMaxPairs];
 };
@@ -48,6 +48,7 @@ struct DecodeParams {
   void* out;             // [B][Hq][d]
   float* partials;       // [B][Hq][n_split][d + 2]
   int batch, hq, hkv, d, n_split;
+  int pairing;           // atf_pairing of the raw queries
   long long n_cache;
   long long kv_len[kMaxDecodeBatch];
   unsigned long long* skipped;  // nullable

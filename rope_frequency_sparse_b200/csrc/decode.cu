@@ -152,8 +152,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const int g = idx / NP, i = idx % NP;
       float r0 = 0.f, r1 = 0.f;
       if (g < G) {
-        const long long e = (static_cast<long long>(b) * p.hq + hk * G + g) * D + 2 * i;
-        const double x0 = __bfloat162float(Q[e]), x1 = __bfloat162float(Q[e + 1]);
+        // dims of pair i: (2i, 2i+1), or (i, i + d/2) for rotate-half queries; the
+        // rotated pair goes to slots (2i, 2i+1), the cache's order
+        const long long row = (static_cast<long long>(b) * p.hq + hk * G + g) * D;
+        const long long ea = row + (p.pairing ? i : 2 * i), eb = ea + (p.pairing ? D / 2 : 1);
+        const double x0 = __bfloat162float(Q[ea]), x1 = __bfloat162float(Q[eb]);
         double sn, cs;
         sincos(static_cast<double>(qpos) * p.omega[i], &sn, &cs);
         r0 = static_cast<float>(x0 * cs - x1 * sn);

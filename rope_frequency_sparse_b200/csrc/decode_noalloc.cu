@@ -59,8 +59,8 @@ extern "C" size_t atf_decode_noalloc_scratch_bytes(void) { return kDecodeScratch
 
 extern "C" atf_status atf_decode_noalloc(const void* q, const void* k_chunked, const void* v, void* out, int batch,
                                          const long long* kv_len, long long n_cache, int heads, int kv_heads, int d,
-                                         double theta, double alpha, unsigned long long* skipped_pairs,
-                                         void* stream) {
+                                         double theta, double alpha, int pairing,
+                                         unsigned long long* skipped_pairs, void* stream) {
   if (batch > 0 && !kv_len) return atf::report_error(ATF_ERR_INVALID_ARG, "decode_noalloc: kv_len is NULL");
   long long max_len = 1;
   for (int b = 0; b < batch; ++b)
@@ -74,6 +74,6 @@ extern "C" atf_status atf_decode_noalloc(const void* q, const void* k_chunked, c
   atf_status st = ATF_OK;
   void* scratch = batch > 0 ? scratch_address(&st) : nullptr;
   if (st != ATF_OK) return st;
-  return atf_decode(q, k_chunked, v, out, batch, kv_len, n_cache, heads, kv_heads, d, theta, alpha, scratch,
-                    kDecodeScratchBytes, skipped_pairs, stream);
+  return atf_decode(q, k_chunked, v, out, batch, kv_len, n_cache, heads, kv_heads, d, theta, alpha, pairing,
+                    scratch, kDecodeScratchBytes, skipped_pairs, stream);
 }

@@ -9,6 +9,12 @@
 // beyond, where an fp32 angle would be off by more than the bf16 step), and the
 // result is rounded once to the output type.
 //
+// Rotate-half checkpoints (NeoX style, e.g. the Qwen2.5 family) pair dims
+// (i, i + d/2) instead.  The attention kernels only ever take dot products of a
+// rotated query with rotated keys, so for them any consistent order of the
+// dimensions is the same: in the rotate-half modes this kernel writes pair i to
+// slots (2i, 2i+1) of its outputs, the interleaved order the kernels read.
+//
 // Pair-chunk-major layout: the decode kernel reads, for far keys, only the
 // low-frequency pairs.  Keys are therefore also written as
 // [batch][head][chunk c = d/16][token][16 elements] so that one chunk of 8
@@ -33,16 +39,27 @@ __global__ void __launch_bounds__(256) rope_kernel(RopeParams p) {
   const int t = static_cast<int>(row % p.seq);
   const int b = static_cast<int>(row / p.seq);
 
+  // dims of pair i in the input: (2i, 2i+1), or (i, i + d/2) in the rotate-half modes
+  const bool half_pairs = p.rotate >= 2;
   double c = 1.0, s = 0.0;
-  if (p.rotate) {
+  if (p.rotate == 1 || p.rotate == 2) {
     const double phi = static_cast<double>(p.pos_offset + t) * s_omega[i];
     sincos(phi, &s, &c);
   }
   const int nchunk = p.d / 16;
   for (int h = 0; h < p.heads; ++h) {
-    const long long e = (row * p.heads + h) * p.d + 2 * i;  // element index of x_{2i}
+    const long long e = (row * p.heads + h) * p.d + 2 * i;  // output slots (2i, 2i+1)
     double x0, x1;
-    if (p.fp32) {
+    if (half_pairs) {
+      const long long ea = (row * p.heads + h) * p.d + i, eb = ea + p.d / 2;
+      if (p.fp32) {
+        x0 = static_cast<const float*>(p.x)[ea];
+        x1 = static_cast<const float*>(p.x)[eb];
+      } else {
+        x0 = __bfloat162float(static_cast<const __nv_bfloat16*>(p.x)[ea]);
+        x1 = __bfloat162float(static_cast<const __nv_bfloat16*>(p.x)[eb]);
+      }
+    } else if (p.fp32) {
       const float2 v = *reinterpret_cast<const float2*>(static_cast<const float*>(p.x) + e);
       x0 = v.x;
       x1 = v.y;
