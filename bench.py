@@ -468,6 +468,32 @@ def run_extra(args, device, stream, flush_buf, peaks):
                                      "frac": gbs / peaks["hbm_gbs"],
                                      "traffic": recorded_traffic("decode.cu", "decode_1m.md")},
                         "data": "seeded torch CUDA normals (torch.Generator), bf16"}
+
+    # KV-cache append into the same caches: a bulk append of 32768 new tokens per
+    # sequence (varlen positions) and a decode step's one new token per sequence
+    n_bulk = 32768
+    kn = torch.randn((w5.batch * n_bulk, w5.kv_heads, w5.d), generator=g, device=device).to(torch.bfloat16)
+    vn = torch.randn((w5.batch * n_bulk, w5.kv_heads, w5.d), generator=g, device=device).to(torch.bfloat16)
+    pos_bulk = [0, N // 3, N // 2, N - n_bulk][: w5.batch]
+
+    def app(ev, n, pos):
+        if ev:
+            ev[0].record(stream)
+        atf.atf_kv_append(kn, vn, kc, v5, w5.batch, [n] * w5.batch, pos, N, w5.kv_heads, w5.d, w5.theta, 0, s)
+        if ev:
+            ev[1].record(stream)
+
+    ev6 = time_steps(lambda ev: app(ev, n_bulk, pos_bulk), 10, 3, stream, flush_buf, n_events=2)
+    ms6 = sum(e[0].elapsed_time(e[1]) for e in ev6) / 10
+    bytes6 = 4 * w5.batch * n_bulk * w5.kv_heads * w5.d * 2  # read k, v; write both caches
+    ev7 = time_steps(lambda ev: app(ev, 1, [N - 1] * w5.batch), 10, 3, stream, flush_buf, n_events=2)
+    us7 = sum(e[0].elapsed_time(e[1]) for e in ev7) / 10 * 1e3
+    out["kv_append"] = {"GBps_bulk": bytes6 / (ms6 * 1e-3) / 1e9, "ms_bulk": ms6,
+                        "bulk": f"{w5.batch} sequences x {n_bulk} new tokens, 28/4 heads, d=128",
+                        "roofline": {"bound": "hbm", "achieved": bytes6 / (ms6 * 1e-3) / 1e9,
+                                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                     "frac": bytes6 / (ms6 * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+                        "us_decode_step_append": us7}
     atf.atf_check(s)
     return out
 

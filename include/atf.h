@@ -168,6 +168,27 @@ atf_status atf_decode_noalloc(const void* q, const void* k_chunked, const void* 
 /* Size in bytes of atf_decode_noalloc's fixed device scratch array. */
 size_t atf_decode_noalloc_scratch_bytes(void);
 
+/* KV-cache append for a varlen batch: the step on either side of the decode
+ * attention ("Was ATFlash anders macht": the decode side reads the rotated key
+ * cache).  New tokens' keys are rotated at their positions and written into the
+ * pair-chunk-major key cache atf_decode reads; their values are copied into the
+ * token-major value cache.
+ *   k_new, v_new:    [total_new][kv_heads][d] bf16: the new tokens of sequence 0,
+ *                    then those of sequence 1, ... (total_new = sum of n_new).
+ *   n_new:           HOST array, batch entries >= 0: new tokens of each sequence.
+ *   pos:             HOST array, batch entries >= 0: position of sequence b's first
+ *                    new token; its tokens take positions (and cache slots)
+ *                    pos[b] .. pos[b] + n_new[b] - 1, with pos[b] + n_new[b] <= n_cache.
+ *   k_cache_chunked: [batch][kv_heads][d/16][n_cache][16] bf16 (atf_rope_layout's
+ *                    chunk-major layout, pairs in the interleaved order).
+ *   v_cache:         [batch][n_cache][kv_heads][d] bf16.
+ *   pairing:         atf_pairing of k_new.
+ * Only the appended slots are written.  Rotation in fp64, one rounding to bf16
+ * (the same values atf_rope_layout produces for those positions). */
+atf_status atf_kv_append(const void* k_new, const void* v_new, void* k_cache_chunked, void* v_cache, int batch,
+                         const int* n_new, const long long* pos, long long n_cache, int kv_heads, int d,
+                         double theta, int pairing, void* stream);
+
 /* Synchronises `stream` and reports ATF_ERR_TIMEOUT if any kernel of this
  * library on the current device gave up a bounded wait since the last
  * atf_check (the device error word is cleared), ATF_ERR_CUDA on a CUDA error. */

@@ -68,6 +68,7 @@ def load_library(path: str = LIB_PATH):
         "atf_decode_workspace_bytes": ([i, i, i, ll, i], sz),
         "atf_decode_noalloc": ([vp, vp, vp, vp, i, vp, ll, i, i, i, d, d, i, vp, vp], i),
         "atf_decode_noalloc_scratch_bytes": ([], sz),
+        "atf_kv_append": ([vp, vp, vp, vp, i, vp, vp, ll, i, i, d, i, vp], i),
         "atf_check": ([vp], i),
         "atf_selftest_timeout": ([ll, vp], i),
         "atf_last_error": ([], ctypes.c_char_p),
@@ -172,6 +173,15 @@ def atf_decode_noalloc_scratch_bytes() -> int:
 
 def atf_decode_workspace_bytes(batch, heads, kv_heads, max_kv_len, d) -> int:
     return int(load_library().atf_decode_workspace_bytes(batch, heads, kv_heads, int(max_kv_len), d))
+
+
+def atf_kv_append(k_new, v_new, k_cache_chunked, v_cache, batch, n_new, pos, n_cache, kv_heads, d, theta,
+                  pairing=ATF_PAIRS_INTERLEAVED, stream=None):
+    nn = np.ascontiguousarray(np.asarray(n_new, dtype=np.int32).reshape(-1))
+    ps = np.ascontiguousarray(np.asarray(pos, dtype=np.int64).reshape(-1))
+    _check(load_library().atf_kv_append(_ptr(k_new), _ptr(v_new), _ptr(k_cache_chunked), _ptr(v_cache), batch,
+                                        nn.ctypes.data_as(ctypes.c_void_p), ps.ctypes.data_as(ctypes.c_void_p),
+                                        int(n_cache), kv_heads, d, float(theta), int(pairing), _stream(stream)))
 
 
 def atf_check(stream=None):

@@ -404,6 +404,55 @@ atf_status atf_decode(const void* q, const void* k_chunked, const void* v, void*
   return ATF_OK;
 }
 
+atf_status atf_kv_append(const void* k_new, const void* v_new, void* k_cache_chunked, void* v_cache, int batch,
+                         const int* n_new, const long long* pos, long long n_cache, int kv_heads, int d,
+                         double theta, int pairing, void* stream) {
+  if (atf_status st = check_params(d, theta, 1.0)) return st;
+  if (batch < 0 || kv_heads < 1 || n_cache < 1) return fail(ATF_ERR_INVALID_ARG, "kv_append: bad sizes");
+  if (n_cache > 0x7fffffffLL) return fail(ATF_ERR_UNSUPPORTED, "kv_append: cache longer than 2^31-1");
+  if (pairing != ATF_PAIRS_INTERLEAVED && pairing != ATF_PAIRS_ROTATE_HALF)
+    return fail(ATF_ERR_INVALID_ARG, "kv_append: pairing %d", pairing);
+  if (batch == 0) return ATF_OK;
+  if (!n_new || !pos) return fail(ATF_ERR_INVALID_ARG, "kv_append: null n_new / pos");
+  long long total = 0;
+  for (int b = 0; b < batch; ++b) {
+    if (n_new[b] < 0 || pos[b] < 0 || pos[b] + n_new[b] > n_cache)
+      return fail(ATF_ERR_INVALID_ARG, "kv_append: sequence %d: %d tokens at %lld do not fit %lld slots", b,
+                  n_new[b], pos[b], n_cache);
+    total += n_new[b];
+  }
+  if (total == 0) return ATF_OK;
+  if (!k_new || !v_new || !k_cache_chunked || !v_cache) return fail(ATF_ERR_INVALID_ARG, "kv_append: null pointer");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache_chunked) || !aligned16(v_cache))
+    return fail(ATF_ERR_INVALID_ARG, "kv_append: pointers must be 16-byte aligned");
+  AppendParams p{};
+  Windows w;
+  kernel_windows(d, theta, INFINITY, &w, p.omega);
+  p.hkv = kv_heads;
+  p.d = d;
+  p.pairing = pairing;
+  p.n_cache = n_cache;
+  const size_t row_bytes = static_cast<size_t>(kv_heads) * d * 2;  // one token of k_new / v_new
+  long long row0 = 0;                                                // first row of the group
+  for (int b0 = 0; b0 < batch; b0 += kMaxDecodeBatch) {
+    const int nb = batch - b0 < kMaxDecodeBatch ? batch - b0 : kMaxDecodeBatch;
+    p.batch = nb;
+    p.cu[0] = 0;
+    for (int i = 0; i < nb; ++i) {
+      p.cu[i + 1] = p.cu[i] + n_new[b0 + i];
+      p.pos[i] = pos[b0 + i];
+    }
+    p.k_new = static_cast<const char*>(k_new) + static_cast<size_t>(row0) * row_bytes;
+    p.v_new = static_cast<const char*>(v_new) + static_cast<size_t>(row0) * row_bytes;
+    p.kc = static_cast<char*>(k_cache_chunked) + static_cast<size_t>(b0) * n_cache * row_bytes;
+    p.vc = static_cast<char*>(v_cache) + static_cast<size_t>(b0) * n_cache * row_bytes;
+    cudaError_t e = launch_kv_append(p, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kv_append kernel launch");
+    row0 += p.cu[nb];
+  }
+  return ATF_OK;
+}
+
 atf_status atf_check(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");

@@ -57,8 +57,21 @@ struct DecodeParams {
   double omega[kMaxPairs];
 };
 
+struct AppendParams {
+  const void* k_new;  // [total_new][hkv][d] bf16, sequences one after the other
+  const void* v_new;  // same layout
+  void* kc;           // rotated key cache, chunk-major [B][Hkv][d/16][n_cache][16]
+  void* vc;           // value cache [B][n_cache][Hkv][d]
+  int batch, hkv, d, pairing;
+  long long n_cache;
+  long long cu[kMaxDecodeBatch + 1];  // first row of sequence b in k_new / v_new
+  long long pos[kMaxDecodeBatch];     // position (cache slot) of sequence b's first new token
+  double omega[kMaxPairs];
+};
+
 // Launchers (return cudaGetLastError() of the launch).
 cudaError_t launch_rope(const RopeParams& p, cudaStream_t s);
+cudaError_t launch_kv_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillParams& p, cudaStream_t s);
 cudaError_t launch_prefill_tc(const PrefillParams& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                               const CUtensorMap& tm_v, bool dense, cudaStream_t s);

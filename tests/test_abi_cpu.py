@@ -81,6 +81,17 @@ def test_rejects_bad_arguments_before_any_device_call(lib):
         atf.ATF_ERR_INVALID_ARG  # workspace too small
     assert _status(lambda: atf.atf_rope_layout(fake, None, fake, 1, 8, 4, 128, 0, 1e7, 1, atf.ATF_FP32)) == \
         atf.ATF_ERR_UNSUPPORTED  # chunk-major is bf16 only
+    assert _status(lambda: atf.atf_rope_layout(fake, fake, None, 1, 8, 4, 128, 0, 1e7, 4, atf.ATF_BF16)) == \
+        atf.ATF_ERR_INVALID_ARG  # no such rotate mode
+    assert _status(lambda: D(fake, fake, fake, fake, 1, [8], 8, 28, 4, 128, 1e7, 1.0, fake, 1 << 20,
+                             pairing=2)) == atf.ATF_ERR_INVALID_ARG  # no such pairing
+    A = atf.atf_kv_append
+    assert _status(lambda: A(fake, fake, fake, fake, 2, [3, 4], [0, 5], 8, 4, 128, 1e7)) == \
+        atf.ATF_ERR_INVALID_ARG  # 5 + 4 > 8 slots
+    assert _status(lambda: A(fake, fake, fake, fake, 1, [-1], [0], 8, 4, 128, 1e7)) == atf.ATF_ERR_INVALID_ARG
+    assert _status(lambda: A(fake + 8, fake, fake, fake, 1, [1], [0], 8, 4, 128, 1e7)) == \
+        atf.ATF_ERR_INVALID_ARG  # misaligned
+    assert _status(lambda: A(fake, fake, fake, fake, 1, [1], [0], 8, 4, 96, 1e7)) == atf.ATF_ERR_UNSUPPORTED
 
 
 def test_empty_inputs_are_no_ops(lib):
@@ -88,6 +99,8 @@ def test_empty_inputs_are_no_ops(lib):
     atf.atf_prefill_ex(None, None, None, None, 0, 16, 16, 28, 4, 128, 0, 0, 1, 1e7, 1.0)
     atf.atf_decode(None, None, None, None, 0, [], 8, 28, 4, 128, 1e7, 1.0, None, 0)
     atf.atf_rope_layout(None, None, None, 0, 8, 4, 128, 0, 1e7, 1, 0)
+    atf.atf_kv_append(None, None, None, None, 0, [], [], 8, 4, 128, 1e7)
+    atf.atf_kv_append(None, None, None, None, 2, [0, 0], [3, 8], 8, 4, 128, 1e7)  # nothing to append
 
 
 def test_workspace_sizes(lib):
