@@ -314,28 +314,36 @@ def run_ours(args, rank, world, local_rank):
     per_alpha["1.0"] = {"tflops": eff / (ms_step * 1e-3) / 1e12, "ms": ms_step}
     per_alpha["inf"] = {"tflops": dense_flops / (ms_dense * 1e-3) / 1e12, "ms": ms_dense}
 
-    # ---- end to end through the C ABI from pinned host buffers
+    # ---- end to end through the C ABI from pinned host buffers: atf_prefill_host
+    # uploads q, k, v, runs RoPE + the windowed prefill and downloads the output,
+    # the copies overlapped with each other and with the kernels
     q_h, k_h, v_h = (t.pin_memory() for t in step.host)
     out_h = torch.empty_like(q_h).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
     d2h = out_h.numel() * out_h.element_size()
+    B, S, Hq, d = step.q.shape
+    Hkv = step.k.shape[2]
+    hws_bytes = atf.atf_prefill_host_workspace_bytes(B, S, S, Hq, Hkv, d, 0)
+    hws = torch.empty(hws_bytes, dtype=torch.uint8, device=device)
 
-    def e2e_step(ev):
+    def e2e_step(ev, chunk_rows=0):
         if ev:
             ev[0].record(stream)
-        step.q.copy_(q_h, non_blocking=True)
-        step.k.copy_(k_h, non_blocking=True)
-        step.v.copy_(v_h, non_blocking=True)
-        B, S, Hq, d = step.q.shape
-        atf.atf_prefill_ex(step.q, step.k, step.v, step.out, B, S, S, Hq, step.k.shape[2], d, 0, atf.ATF_BF16, 0,
-                           w.theta, 1.0, None, step.ws, step.ws_bytes, s)
-        out_h.copy_(step.out, non_blocking=True)
+        atf.atf_prefill_host(q_h, k_h, v_h, out_h, B, S, S, Hq, Hkv, d, 0, 0, w.theta, 1.0, hws, hws_bytes,
+                             chunk_rows, None, s)
         if ev:
             ev[1].record(stream)
 
     evs_e = time_steps(e2e_step, args.steps, args.warmup, stream, flush_buf, n_events=2)
     ms_e2e = dist_max(sum(e[0].elapsed_time(e[1]) for e in evs_e) / args.steps)
     e2e_val = world * eff / (ms_e2e * 1e-3) / 1e12
+    atf.atf_check(s)
+    e2e_sweep = {}
+    if world == 1 and not args.no_extra:
+        for rows in (512, 1024, 2048, S):
+            ev_c = time_steps(lambda ev: e2e_step(ev, rows), max(3, args.steps // 2), 1, stream, flush_buf,
+                              n_events=2)
+            e2e_sweep[str(rows)] = sum(e[0].elapsed_time(e[1]) for e in ev_c) / len(ev_c)
 
     extra = {}
     if world == 1 and not args.no_extra:
@@ -359,8 +367,10 @@ def run_ours(args, rank, world, local_rank):
                      "kernel": "prefill_tc_kernel<128,sparse>", "peak_kind": f"{peak_kind} bf16 burst",
                      "kernel_ms": ms_kern},
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": ms_e2e},
-        "gpu_launches": 3 * args.steps,
+                "ms_per_step": ms_e2e,
+                "call": "atf_prefill_host (pinned host buffers, default chunk schedule, two compute streams)",
+                "ms_by_chunk_rows": e2e_sweep},
+        "gpu_launches": 3 * args.steps,  # rope(q), rope(k), prefill per step of the device-resident timing
         "clocks": clocks.summary(),
         "wall_s_timed_region": t_wall,
     }

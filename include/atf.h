@@ -117,6 +117,34 @@ atf_status atf_prefill_ex(const atf_prefill_args* args, void* stream);
 atf_status atf_prefill(const void* q, const void* k, const void* v, void* out, int seq, int heads, int kv_heads,
                        int d, double theta, double alpha, void* stream);
 
+/* Device scratch bytes atf_prefill_host needs: device copies of q, k, v, their
+ * rotated forms (not when rotated) and the output. */
+size_t atf_prefill_host_workspace_bytes(int batch, int q_len, int kv_len, int heads, int kv_heads, int d,
+                                        int rotated);
+
+/* Prefill from host memory: the same operation and result as atf_prefill_ex on
+ * device copies of the inputs, with the host<->device copies overlapped with
+ * each other and with the kernels.
+ *   args->q, k, v, out: HOST memory, shapes as in atf_prefill_ex.  Page-locked
+ *       memory (cudaHostAlloc / cudaHostRegister) lets the copies overlap;
+ *       pageable memory gives the same result with the copies serialised.
+ *   args->workspace: DEVICE scratch of atf_prefill_host_workspace_bytes(...)
+ *       bytes, 16-byte aligned.
+ *   args->dtype: ATF_BF16 only (else ATF_ERR_UNSUPPORTED).
+ *   args->skipped_pairs: device pointer or NULL, as in atf_prefill_ex.
+ *   chunk_rows: query rows per pipeline chunk (> 0), or 0 for q_len / 8
+ *       rounded up to a multiple of 256.
+ * Work order: k and v are uploaded whole, then the query rows chunk by chunk
+ * from the last chunk to the first; each chunk is rotated and attended (as a
+ * chunked prefill at offset q_offset + first row of the chunk, on `stream`) as
+ * soon as it is on the device, and its output rows are downloaded while later
+ * chunks run.  The copies run on two streams the library creates once per
+ * device and host thread; before returning, the call makes `stream` wait for
+ * both, so `out` holds the result once `stream` has reached that point
+ * (synchronise `stream` before reading it).  The same workspace must not be in
+ * use by another call that may run concurrently. */
+atf_status atf_prefill_host(const atf_prefill_args* args, int chunk_rows, void* stream);
+
 /* Decode: one new query per sequence against a rotated key cache.
  *   q:          [batch][heads][d] bf16, NOT rotated; rotated here at position kv_len[b]-1
  *               with the given atf_pairing.

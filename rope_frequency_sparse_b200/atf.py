@@ -64,6 +64,8 @@ def load_library(path: str = LIB_PATH):
         "atf_prefill_workspace_bytes": ([i, i, i, i, i, i, i, i], sz),
         "atf_prefill_ex": ([ctypes.POINTER(PrefillArgs), vp], i),
         "atf_prefill": ([vp, vp, vp, vp, i, i, i, i, d, d, vp], i),
+        "atf_prefill_host_workspace_bytes": ([i, i, i, i, i, i, i], sz),
+        "atf_prefill_host": ([ctypes.POINTER(PrefillArgs), i, vp], i),
         "atf_decode": ([vp, vp, vp, vp, i, vp, ll, i, i, i, d, d, i, vp, sz, vp, vp], i),
         "atf_decode_workspace_bytes": ([i, i, i, ll, i], sz),
         "atf_decode_noalloc": ([vp, vp, vp, vp, i, vp, ll, i, i, i, d, d, i, vp, vp], i),
@@ -141,6 +143,20 @@ def atf_prefill_ex(q, k, v, out, batch, q_len, kv_len, heads, kv_heads, d, q_off
                     int(dtype), int(rotated), float(theta), float(alpha), _ptr(skipped_pairs), _ptr(workspace),
                     int(workspace_bytes), int(pairing))
     _check(load_library().atf_prefill_ex(ctypes.byref(a), _stream(stream)))
+
+
+def atf_prefill_host_workspace_bytes(batch, q_len, kv_len, heads, kv_heads, d, rotated) -> int:
+    return int(load_library().atf_prefill_host_workspace_bytes(batch, q_len, kv_len, heads, kv_heads, d, rotated))
+
+
+def atf_prefill_host(q, k, v, out, batch, q_len, kv_len, heads, kv_heads, d, q_offset, rotated, theta, alpha,
+                     workspace, workspace_bytes, chunk_rows=0, skipped_pairs=None, stream=None,
+                     pairing=ATF_PAIRS_INTERLEAVED):
+    """q, k, v, out are host buffers (CPU tensors, pinned for overlap); workspace is device memory."""
+    a = PrefillArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(out), batch, q_len, kv_len, heads, kv_heads, d, int(q_offset),
+                    ATF_BF16, int(rotated), float(theta), float(alpha), _ptr(skipped_pairs), _ptr(workspace),
+                    int(workspace_bytes), int(pairing))
+    _check(load_library().atf_prefill_host(ctypes.byref(a), int(chunk_rows), _stream(stream)))
 
 
 def atf_prefill(q, k, v, out, seq, heads, kv_heads, d, theta, alpha, stream=None):
@@ -223,6 +239,30 @@ def prefill(q, k, v, theta, alpha, q_offset=0, rotated=False, skipped=None, out=
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     atf_prefill_ex(q, k, v, out, B, q_len, kv_len, Hq, Hkv, d, q_offset, dt, int(rotated), theta, alpha,
                    skipped, workspace, need, stream, pairing)
+    return out
+
+
+def prefill_host(q, k, v, theta, alpha, q_offset=0, rotated=False, skipped=None, out=None, workspace=None,
+                 chunk_rows=0, stream=None, pairing=ATF_PAIRS_INTERLEAVED, device=None):
+    """Windowed causal prefill of host tensors (CPU, bf16; pinned for overlapped
+    copies): q [B][q_len][Hq][d], k/v [B][kv_len][Hkv][d].  Returns the host
+    output once the stream has finished (this call synchronises the stream)."""
+    import torch
+
+    B, q_len, Hq, d = q.shape
+    _, kv_len, Hkv, _ = k.shape
+    for t in (q, k, v):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise TypeError("prefill_host takes contiguous bf16 CPU tensors")
+    if out is None:
+        out = torch.empty_like(q, pin_memory=q.is_pinned())
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    need = atf_prefill_host_workspace_bytes(B, q_len, kv_len, Hq, Hkv, d, int(rotated))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    atf_prefill_host(q, k, v, out, B, q_len, kv_len, Hq, Hkv, d, q_offset, int(rotated), theta, alpha, workspace,
+                     need, chunk_rows, skipped, stream, pairing)
+    atf_check(stream)
     return out
 
 

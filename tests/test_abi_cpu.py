@@ -92,6 +92,27 @@ def test_rejects_bad_arguments_before_any_device_call(lib):
     assert _status(lambda: A(fake + 8, fake, fake, fake, 1, [1], [0], 8, 4, 128, 1e7)) == \
         atf.ATF_ERR_INVALID_ARG  # misaligned
     assert _status(lambda: A(fake, fake, fake, fake, 1, [1], [0], 8, 4, 96, 1e7)) == atf.ATF_ERR_UNSUPPORTED
+    H = atf.atf_prefill_host
+    need = atf.atf_prefill_host_workspace_bytes(1, 128, 128, 28, 4, 128, 0)
+    assert _status(lambda: H(fake, fake, fake, fake, 1, 128, 128, 28, 4, 128, 0, 0, 1e7, 1.0, fake, need - 1)) == \
+        atf.ATF_ERR_INVALID_ARG  # workspace too small
+    assert "workspace" in atf.atf_last_error()
+    assert _status(lambda: H(fake, fake, fake, fake, 1, 128, 128, 28, 4, 128, 0, 0, 1e7, 1.0, fake + 8, need)) == \
+        atf.ATF_ERR_INVALID_ARG  # misaligned workspace
+    assert _status(lambda: H(fake, fake, fake, fake, 1, 128, 100, 28, 4, 128, 0, 0, 1e7, 1.0, fake, need)) == \
+        atf.ATF_ERR_INVALID_ARG  # kv_len < q_offset + q_len
+    assert _status(lambda: H(fake, fake, fake, fake, 1, 128, 128, 28, 4, 96, 0, 0, 1e7, 1.0, fake, need)) == \
+        atf.ATF_ERR_UNSUPPORTED
+    assert _status(lambda: H(fake, fake, fake, fake, 1, 128, 128, 28, 5, 128, 0, 0, 1e7, 1.0, fake, need)) == \
+        atf.ATF_ERR_INVALID_ARG  # heads % kv_heads
+    assert _status(lambda: H(fake, fake, fake, fake, 1, 128, 128, 28, 4, 128, 0, 0, 1e7, 1.0, fake, need,
+                             chunk_rows=-1)) == atf.ATF_ERR_INVALID_ARG
+    assert _status(lambda: H(fake, fake, fake, fake, 1, 128, 128, 28, 4, 128, 0, 0, 1e7, 1.0, fake, need,
+                             pairing=2)) == atf.ATF_ERR_INVALID_ARG
+    assert _status(lambda: H(fake, None, fake, fake, 1, 128, 128, 28, 4, 128, 0, 0, 1e7, 1.0, fake, need)) == \
+        atf.ATF_ERR_INVALID_ARG
+    assert _status(lambda: H(fake, fake, fake, fake, 1, 128, 128, 28, 4, 128, 0, 0, 0.5, 1.0, fake, need)) == \
+        atf.ATF_ERR_INVALID_ARG  # theta <= 1
 
 
 def test_empty_inputs_are_no_ops(lib):
@@ -101,12 +122,19 @@ def test_empty_inputs_are_no_ops(lib):
     atf.atf_rope_layout(None, None, None, 0, 8, 4, 128, 0, 1e7, 1, 0)
     atf.atf_kv_append(None, None, None, None, 0, [], [], 8, 4, 128, 1e7)
     atf.atf_kv_append(None, None, None, None, 2, [0, 0], [3, 8], 8, 4, 128, 1e7)  # nothing to append
+    atf.atf_prefill_host(None, None, None, None, 1, 0, 0, 28, 4, 128, 0, 0, 1e7, 1.0, None, 0)
 
 
 def test_workspace_sizes(lib):
     assert atf.atf_prefill_workspace_bytes(1, 8192, 8192, 28, 4, 128, 0, 1) == 0
     ws = atf.atf_prefill_workspace_bytes(1, 8192, 8192, 28, 4, 128, 0, 0)
     assert ws >= 8192 * 28 * 128 * 2 + 8192 * 4 * 128 * 2
+    # host path: device copies of q, k, v, rotated q and k, and the output
+    hws = atf.atf_prefill_host_workspace_bytes(2, 1000, 1500, 28, 4, 128, 0)
+    qb, kb = 2 * 1000 * 28 * 128 * 2, 2 * 1500 * 4 * 128 * 2
+    assert hws == 3 * qb + 3 * kb
+    assert atf.atf_prefill_host_workspace_bytes(2, 1000, 1500, 28, 4, 128, 1) == 2 * qb + 2 * kb
+    assert atf.atf_prefill_host_workspace_bytes(0, 1000, 1500, 28, 4, 128, 0) == 0
     dws = atf.atf_decode_workspace_bytes(4, 28, 4, 1 << 20, 128)
     assert dws % (4 * 28 * 130 * 4) == 0 and dws > 0
 
