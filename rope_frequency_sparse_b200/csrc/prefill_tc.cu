@@ -62,7 +62,6 @@ constexpr int kRegsSoftmax = 216;  // softmax warpgroups after reallocation
 static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split exceeds the launch");
 constexpr uint32_t kTmemCols = 512;
 constexpr int kStash = 12;        // zeroed query pairs kept per row (more are re-read from global memory)
-constexpr int kTabPairs = 4;      // key pairs converted per batch of boundary corrections
 
 // 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 on [-1/2, 1/2]: coefficients chosen for the
 // smallest maximum relative error (7.5e-5, Lawson's iteratively reweighted least
@@ -95,9 +94,6 @@ struct Shared {
   // Per Q tile, the query pairs most recently zeroed in its shared-memory copy
   // ([slot][row], slot = pair - first zeroed pair), read back by add-back corrections.
   uint32_t stash[NQ][kStash][BM];
-  // Per softmax warp: up to kTabPairs key pairs over a 32-column chunk as fp32,
-  // (k_2i(c), k_2i(c+1), k_2i+1(c), k_2i+1(c+1)) per column pair, for the boundary corrections.
-  float4 ktab[8][kTabPairs][16];
 };
 
 template <int D>
@@ -478,6 +474,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int cen = static_cast<int>(center);
             const int cw = quarter * 32 + cen;  // threshold offset of the warp's first row
             const uint32_t kbase = smem_u32(sK + s * C::TILE_BYTES);
+            const uint32_t q_base = smem_u32(sQg);
+            const uint32_t stash_base = smem_u32(&sh->stash[g][0][r]);
 #pragma unroll 1
             for (int hb = a; hb < u; hb += 32) {
               // classify pair hb + lane: the chunks some row of this warp must
@@ -510,75 +508,56 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                   for (int cc = 0; cc < 32; ++cc) x[cc] = 0.f;
                 }
-                do {
-                  // up to kTabPairs pairs: convert their keys for this chunk, then apply
-                  int kb[kTabPairs];
-                  uint32_t qpb[kTabPairs];
-                  int nb = 0;
-#pragma unroll
-                  for (int b = 0; b < kTabPairs; ++b) {
-                    kb[b] = 0;
-                    qpb[b] = 0u;
-                    if (tbits) {  // warp-uniform
-                      const int k = __ffs(tbits) - 1;
-                      tbits &= tbits - 1;
-                      kb[b] = k;
-                      nb = b + 1;
-                      const int i = hb + k;
-                      const uint32_t kw = lds32(kbase + (i >> 5) * (BN * 128) + (i & 3) * 4 + (c_lo + lane) * 128 +
-                                                ((((i & 31) >> 2) ^ (lane & 7)) << 4));
-                      const uint32_t kn = __shfl_down_sync(0xffffffffu, kw, 1);
-                      if (!(lane & 1))
-                        sh->ktab[warp - 4][b][lane >> 1] =
-                            make_float4(bf16lo_to_f32(kw), bf16lo_to_f32(kn), bf16hi_to_f32(kw), bf16hi_to_f32(kn));
-                      if (row_ok) {
-                        if (i >= z)
-                          qpb[b] = *reinterpret_cast<const uint32_t*>(sQg + pair_offset(r, i));
-                        else if (static_cast<unsigned>(i - zst) < static_cast<unsigned>(kStash))
-                          qpb[b] = sh->stash[g][i - zst][r];
-                        else
-                          qpb[b] = __ldg(qrow + i);
-                      }
-                    }
-                  }
-                  __syncwarp();
+                // Each pair of the chunk in turn.  Its key words (k_2i(c), k_2i+1(c))
+                // for the chunk's 32 columns are read straight from the K tile: the
+                // address depends only on the column, so every lane issues the same
+                // 32 broadcast loads, with no staging and no warp synchronisation.
 #pragma unroll 1
-                  for (int b = 0; b < nb; ++b) {
-                    const int k = b == 0 ? kb[0] : b == 1 ? kb[1] : b == 2 ? kb[2] : kb[3];
-                    const uint32_t qp = b == 0 ? qpb[0] : b == 1 ? qpb[1] : b == 2 ? qpb[2] : qpb[3];
-                    const int i = hb + k;
-                    const int wi = __shfl_sync(0xffffffffu, wl, k);
-                    const bool add = i < z;  // zeroed pair: add back where c >= tl; else subtract where c < tl
-                    const float sg = add ? 1.f : -1.f;
-                    const uint64_t qa2 = pack2(sg * bf16lo_to_f32(qp), sg * bf16lo_to_f32(qp));
-                    const uint64_t qb2 = pack2(sg * bf16hi_to_f32(qp), sg * bf16hi_to_f32(qp));
-                    const float4* tab = sh->ktab[warp - 4][b];
-                    if ((fbits >> k) & 1u) {  // every row of the warp corrects the whole chunk
+                while (tbits) {
+                  const int k = __ffs(tbits) - 1;
+                  tbits &= tbits - 1;
+                  const int i = hb + k;
+                  uint32_t qp = 0u;
+                  if (row_ok) {
+                    if (i >= z)
+                      qp = lds32(q_base + pair_offset(r, i));
+                    else if (static_cast<unsigned>(i - zst) < static_cast<unsigned>(kStash))
+                      qp = lds32(stash_base + static_cast<uint32_t>((i - zst) * BM) * 4u);
+                    else
+                      qp = __ldg(qrow + i);
+                  }
+                  const uint32_t kp = kbase + (i >> 5) * (BN * 128) + c_lo * 128 + (i & 3) * 4;
+                  const uint32_t ci = static_cast<uint32_t>((i & 31) >> 2);
+                  uint32_t kw[32];
 #pragma unroll
-                      for (int cp = 0; cp < 16; ++cp) {
-                        const float4 t = tab[cp];
-                        uint64_t x2 = pack2(x[2 * cp], x[2 * cp + 1]);
-                        x2 = ffma2(qa2, pack2(t.x, t.y), x2);
-                        x2 = ffma2(qb2, pack2(t.z, t.w), x2);
-                        unpack2(x2, x[2 * cp], x[2 * cp + 1]);
-                      }
-                    } else {
-                      const int tc = r + cen - wi - c_lo;  // chunk columns cc < tc lie outside the window
+                  for (int cc = 0; cc < 32; ++cc) kw[cc] = lds32(kp + cc * 128 + ((ci ^ (cc & 7)) << 4));
+                  const int wi = __shfl_sync(0xffffffffu, wl, k);
+                  const bool add = i < z;  // zeroed pair: add back where c >= tl; else subtract where c < tl
+                  const float sg = add ? 1.f : -1.f;
+                  const uint64_t qa2 = pack2(sg * bf16lo_to_f32(qp), sg * bf16lo_to_f32(qp));
+                  const uint64_t qb2 = pack2(sg * bf16hi_to_f32(qp), sg * bf16hi_to_f32(qp));
+                  if ((fbits >> k) & 1u) {  // every row of the warp corrects the whole chunk
 #pragma unroll
-                      for (int cp = 0; cp < 16; ++cp) {
-                        const float4 t = tab[cp];
-                        uint64_t y2 = pack2(x[2 * cp], x[2 * cp + 1]);
-                        y2 = ffma2(qa2, pack2(t.x, t.y), y2);
-                        y2 = ffma2(qb2, pack2(t.z, t.w), y2);
-                        float y0, y1;
-                        unpack2(y2, y0, y1);
-                        if ((2 * cp >= tc) == add) x[2 * cp] = y0;
-                        if ((2 * cp + 1 >= tc) == add) x[2 * cp + 1] = y1;
-                      }
+                    for (int cp = 0; cp < 16; ++cp) {
+                      uint64_t x2 = pack2(x[2 * cp], x[2 * cp + 1]);
+                      x2 = ffma2(qa2, pack2(bf16lo_to_f32(kw[2 * cp]), bf16lo_to_f32(kw[2 * cp + 1])), x2);
+                      x2 = ffma2(qb2, pack2(bf16hi_to_f32(kw[2 * cp]), bf16hi_to_f32(kw[2 * cp + 1])), x2);
+                      unpack2(x2, x[2 * cp], x[2 * cp + 1]);
+                    }
+                  } else {
+                    const int tc = r + cen - wi - c_lo;  // chunk columns cc < tc lie outside the window
+#pragma unroll
+                    for (int cp = 0; cp < 16; ++cp) {
+                      uint64_t y2 = pack2(x[2 * cp], x[2 * cp + 1]);
+                      y2 = ffma2(qa2, pack2(bf16lo_to_f32(kw[2 * cp]), bf16lo_to_f32(kw[2 * cp + 1])), y2);
+                      y2 = ffma2(qb2, pack2(bf16hi_to_f32(kw[2 * cp]), bf16hi_to_f32(kw[2 * cp + 1])), y2);
+                      float y0, y1;
+                      unpack2(y2, y0, y1);
+                      if ((2 * cp >= tc) == add) x[2 * cp] = y0;
+                      if ((2 * cp + 1 >= tc) == add) x[2 * cp + 1] = y1;
                     }
                   }
-                  __syncwarp();
-                } while (tbits);
+                }
                 tmem_st32(s_tmem + c_lo, reinterpret_cast<uint32_t*>(x));
                 s_chunks |= 1u << qc;
               }
