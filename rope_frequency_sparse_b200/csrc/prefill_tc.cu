@@ -476,6 +476,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t kbase = smem_u32(sK + s * C::TILE_BYTES);
             const uint32_t q_base = smem_u32(sQg);
             const uint32_t stash_base = smem_u32(&sh->stash[g][0][r]);
+            // chunks past every row's last valid column (beyond the causal diagonal
+            // or the last key) are masked out whole: nothing there needs correcting
+            const int cmax_w = __reduce_max_sync(0xffffffffu, cmax);
 #pragma unroll 1
             for (int hb = a; hb < u; hb += 32) {
               // classify pair hb + lane: the chunks some row of this warp must
@@ -489,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int qc = 0; qc < BN / 32; ++qc) {
                 const int c_lo = 32 * qc;
-                const bool touch = valid && (addl ? (c_lo + 31 >= twl) : (c_lo < twl + 31));
+                const bool touch = valid && c_lo <= cmax_w && (addl ? (c_lo + 31 >= twl) : (c_lo < twl + 31));
                 const bool fullc = valid && (addl ? (c_lo >= twl + 31) : (c_lo + 31 < twl));
                 tm |= static_cast<uint32_t>(touch) << qc;
                 fm |= static_cast<uint32_t>(fullc) << qc;
