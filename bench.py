@@ -479,6 +479,37 @@ def run_extra(args, device, stream, flush_buf, peaks):
                                      "traffic": recorded_traffic("decode.cu", "decode_1m.md")},
                         "data": "seeded torch CUDA normals (torch.Generator), bf16"}
 
+    # FASA-style decode on the same cache: token scores on the 16 lowest-frequency
+    # pairs (two 8-pair chunks), 2048 keys kept per query head, attention on those
+    mask16, budget = 0xFFFF << 48, 2048
+    fws_b = atf.atf_fasa_workspace_bytes(w5.batch, w5.q_heads, N, budget, w5.d)
+    fws = torch.empty(fws_b, dtype=torch.uint8, device=device)
+
+    def fas(ev):
+        if ev:
+            ev[0].record(stream)
+        atf.atf_fasa_decode(q5, kc, v5, o5, w5.batch, kv_len, N, w5.q_heads, w5.kv_heads, w5.d, mask16, budget,
+                            None, None, fws, fws_b, s)
+        if ev:
+            ev[1].record(stream)
+
+    ev8 = time_steps(fas, 10, 3, stream, flush_buf, n_events=2)
+    ms8 = sum(e[0].elapsed_time(e[1]) for e in ev8) / 10
+    # algorithmic bytes: the dominant pairs of every key (4 B per pair, key and kv
+    # head), the kept keys' K and V rows, q and out; "moved" adds the fp32 scores
+    # written by the scoring kernel and read back by the selection
+    alg8 = (w5.batch * w5.kv_heads * N * 16 * 4 + w5.batch * w5.q_heads * budget * w5.d * 2 * 2
+            + 2 * w5.batch * w5.q_heads * w5.d * 2)
+    moved8 = alg8 + 2 * w5.batch * w5.q_heads * N * 4
+    gbs8 = alg8 / (ms8 * 1e-3) / 1e9
+    out["fasa_1m"] = {"ms": ms8, "speedup_vs_windowed_decode": ms5 / ms8, "speedup_vs_dense_decode": ms5d / ms8,
+                      "GBps_algorithmic": gbs8, "GBps_moved": moved8 / (ms8 * 1e-3) / 1e9,
+                      "algorithmic_bytes": alg8, "moved_bytes": moved8,
+                      "config": f"{w5.batch} x {N} cached keys, 28/4 heads, d=128, 16 dominant pairs, "
+                                f"budget {budget} keys per query head",
+                      "roofline": {"bound": "hbm", "achieved": gbs8, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                   "frac": gbs8 / peaks["hbm_gbs"]}}
+
     # KV-cache append into the same caches: a bulk append of 32768 new tokens per
     # sequence (varlen positions) and a decode step's one new token per sequence
     n_bulk = 32768

@@ -217,6 +217,41 @@ atf_status atf_kv_append(const void* k_new, const void* v_new, void* k_cache_chu
                          const int* n_new, const long long* pos, long long n_cache, int kv_heads, int d,
                          double theta, int pairing, void* stream);
 
+/* FASA-style decode (page "FASA", section "Das FASA-Framework arbeitet in zwei
+ * Hauptphasen"): a token importance predictor scores every cached key on a given
+ * set of dominant RoPE frequency pairs, each query head keeps its `budget`
+ * best keys, and attention runs over those keys only.
+ *   q_rot:     [batch][heads][d] bf16, ALREADY rotated at the query's position
+ *              (e.g. by atf_rope_layout), pairs interleaved.
+ *   k_chunked: [batch][kv_heads][d/16][n_cache][16] bf16 rotated key cache (the
+ *              layout atf_decode reads); v: [batch][n_cache][kv_heads][d] bf16.
+ *   kv_len:    HOST array, batch entries in [1, n_cache]: keys 0..kv_len[b]-1.
+ *   pair_mask: bit i set = pair i (dims 2i, 2i+1) is dominant; non-empty, bits
+ *              below d/2 only.  Only the 8-pair cache chunks holding a dominant
+ *              pair are read for the scores.
+ *   budget:    keys kept per query head, 1..4096 (all keys when kv_len <= budget).
+ * Score of key n for query head h: from +0, every dim j of the dominant pairs
+ * in ascending order (2i, then 2i+1) adds its product with one fp32 fused
+ * multiply-add, s <- fl(q_j k_j + s); -0 counts as +0.  The kept
+ * keys are the `budget` highest scores, equal scores by lower index.  Output:
+ * out[b][h] = softmax over the kept keys of (1/sqrt d) q.k (all d dims), times
+ * their values, bf16.
+ *   selected:  device int32 [batch][heads][budget] or NULL: the kept key indices,
+ *              ascending, -1 past min(kv_len, budget).
+ *   scores:    device fp32 [batch][heads][n_cache] or NULL: the scores (entries
+ *              n >= kv_len[b] are not written).
+ *   workspace: device scratch of atf_fasa_workspace_bytes(...) bytes (the
+ *              sizes assume selected and scores are NULL; less is needed when
+ *              they are given).
+ * Errors: d not 64/128, more than 8 query heads per kv head, batch above 64,
+ * budget outside [1, 4096] -> ATF_ERR_UNSUPPORTED; bad sizes, mask or kv_len,
+ * small workspace, null or misaligned pointers -> ATF_ERR_INVALID_ARG. */
+atf_status atf_fasa_decode(const void* q_rot, const void* k_chunked, const void* v, void* out, int batch,
+                           const long long* kv_len, long long n_cache, int heads, int kv_heads, int d,
+                           unsigned long long pair_mask, int budget, int* selected, float* scores,
+                           void* workspace, size_t workspace_bytes, void* stream);
+size_t atf_fasa_workspace_bytes(int batch, int heads, long long n_cache, int budget, int d);
+
 /* Synchronises `stream` and reports ATF_ERR_TIMEOUT if any kernel of this
  * library on the current device gave up a bounded wait since the last
  * atf_check (the device error word is cleared), ATF_ERR_CUDA on a CUDA error. */

@@ -19,10 +19,15 @@ Readings of what the page leaves open (each also listed in the design doc):
   keys and their values.
 
 The selection is an integer decision taken on floating-point scores, so both
-sides take it on the same fp32 numbers: each pair's contribution is
-fl(fl(qa*ka) + fl(qb*kb)) (a bf16 x bf16 product is exact in fp32), and the
-pair contributions are summed one by one in ascending pair order with fp32
-round-to-nearest additions (no fused multiply-add).  FAC itself is fp64.
+sides take it on the same fp32 numbers: starting from +0, the dims of the
+dominant pairs are taken in ascending order (2i, then 2i+1, pairs ascending)
+and each adds its product with one fused multiply-add in fp32,
+s <- fl(q_j * k_j + s).  Here that rounding is reproduced in fp64: q_j * k_j (a
+bf16 x bf16 product, 16 significant bits) and s (24 bits) sum exactly in fp64
+whenever their exponents are within 28 of each other; otherwise the smaller
+term is below a quarter of an fp32 ulp of the larger, which is itself an fp32
+number, and both roundings return it.  So fp32(fp64(s) + fp64(q_j) * fp64(k_j))
+is exactly the fused result.  FAC itself is fp64.
 
 Pins (tests/test_fasa_oracle_cpu.py): the all-pairs score equals the full dot
 product within fp32 summation error; a one-pair score equals that pair's
@@ -80,14 +85,10 @@ def tip_scores(q_rot, k_rot, kv_len, mask: int) -> np.ndarray:
         L = int(kl[b])
         for h in range(Hq):
             kk = k[b, :L, h // G, :]  # [L][d]
-            s = None
+            s = np.zeros(L, dtype=np.float32)
             for i in pairs:
-                pa = q[b, h, 2 * i] * kk[:, 2 * i]          # exact in fp32
-                pb = q[b, h, 2 * i + 1] * kk[:, 2 * i + 1]  # exact in fp32
-                t = (pa + pb).astype(np.float32)            # one rounding
-                s = t if s is None else (s + t).astype(np.float32)
-            if s is None:
-                s = np.zeros(L, dtype=np.float32)
+                for j in (2 * i, 2 * i + 1):  # one fused multiply-add per dim
+                    s = (s.astype(np.float64) + np.float64(q[b, h, j]) * kk[:, j].astype(np.float64)).astype(np.float32)
             out[b, h, :L] = s + np.float32(0.0)  # -0 and +0 score alike
     return out
 

@@ -71,6 +71,8 @@ def load_library(path: str = LIB_PATH):
         "atf_decode_noalloc": ([vp, vp, vp, vp, i, vp, ll, i, i, i, d, d, i, vp, vp], i),
         "atf_decode_noalloc_scratch_bytes": ([], sz),
         "atf_kv_append": ([vp, vp, vp, vp, i, vp, vp, ll, i, i, d, i, vp], i),
+        "atf_fasa_decode": ([vp, vp, vp, vp, i, vp, ll, i, i, i, ctypes.c_ulonglong, i, vp, vp, vp, sz, vp], i),
+        "atf_fasa_workspace_bytes": ([i, i, ll, i, i], sz),
         "atf_check": ([vp], i),
         "atf_selftest_timeout": ([ll, vp], i),
         "atf_last_error": ([], ctypes.c_char_p),
@@ -200,6 +202,19 @@ def atf_kv_append(k_new, v_new, k_cache_chunked, v_cache, batch, n_new, pos, n_c
                                         int(n_cache), kv_heads, d, float(theta), int(pairing), _stream(stream)))
 
 
+def atf_fasa_workspace_bytes(batch, heads, n_cache, budget, d) -> int:
+    return int(load_library().atf_fasa_workspace_bytes(batch, heads, int(n_cache), budget, d))
+
+
+def atf_fasa_decode(q_rot, k_chunked, v, out, batch, kv_len, n_cache, heads, kv_heads, d, pair_mask, budget,
+                    selected=None, scores=None, workspace=None, workspace_bytes=0, stream=None):
+    kl = np.ascontiguousarray(np.asarray(kv_len, dtype=np.int64).reshape(-1))
+    _check(load_library().atf_fasa_decode(_ptr(q_rot), _ptr(k_chunked), _ptr(v), _ptr(out), batch,
+                                          kl.ctypes.data_as(ctypes.c_void_p), int(n_cache), heads, kv_heads, d,
+                                          int(pair_mask) & ((1 << 64) - 1), int(budget), _ptr(selected),
+                                          _ptr(scores), _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
 def atf_check(stream=None):
     _check(load_library().atf_check(_stream(stream)))
 
@@ -280,6 +295,24 @@ def decode(q, k_chunked, v, kv_len, theta, alpha, skipped=None, out=None, worksp
     if out is None:
         out = torch.empty_like(q)
     atf_decode(q, k_chunked, v, out, B, kl, N, Hq, Hkv, d, theta, alpha, workspace, need, skipped, stream, pairing)
+    return out
+
+
+def fasa_decode(q_rot, k_chunked, v, kv_len, pair_mask, budget, selected=None, scores=None, out=None,
+                workspace=None, stream=None):
+    """FASA-style decode; q_rot [B][Hq][d] (rotated), k_chunked [B][Hkv][d/16][N][16],
+    v [B][N][Hkv][d] (torch, CUDA, bf16).  Returns out [B][Hq][d]."""
+    import torch
+
+    B, Hq, d = q_rot.shape
+    _, Hkv, _, N, _ = k_chunked.shape
+    if out is None:
+        out = torch.empty_like(q_rot)
+    need = atf_fasa_workspace_bytes(B, Hq, N, budget, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_rot.device)
+    atf_fasa_decode(q_rot, k_chunked, v, out, B, kv_len, N, Hq, Hkv, d, pair_mask, budget, selected, scores,
+                    workspace, need, stream)
     return out
 
 

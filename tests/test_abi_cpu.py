@@ -92,6 +92,28 @@ def test_rejects_bad_arguments_before_any_device_call(lib):
     assert _status(lambda: A(fake + 8, fake, fake, fake, 1, [1], [0], 8, 4, 128, 1e7)) == \
         atf.ATF_ERR_INVALID_ARG  # misaligned
     assert _status(lambda: A(fake, fake, fake, fake, 1, [1], [0], 8, 4, 96, 1e7)) == atf.ATF_ERR_UNSUPPORTED
+    F = atf.atf_fasa_decode
+    fws = atf.atf_fasa_workspace_bytes(1, 28, 64, 16, 128)
+    ok_args = dict(batch=1, kv_len=[64], n_cache=64, heads=28, kv_heads=4, d=128, pair_mask=0xFF, budget=16)
+
+    def fasa(**kw):
+        a = dict(ok_args, **kw)
+        return _status(lambda: F(fake, fake, fake, fake, a["batch"], a["kv_len"], a["n_cache"], a["heads"],
+                                 a["kv_heads"], a["d"], a["pair_mask"], a["budget"], workspace=kw.get("ws", fake),
+                                 workspace_bytes=kw.get("wsb", fws)))
+
+    assert fasa(pair_mask=0) == atf.ATF_ERR_INVALID_ARG
+    assert fasa(d=64, pair_mask=1 << 32) == atf.ATF_ERR_INVALID_ARG  # pair past d/2
+    assert fasa(budget=0) == atf.ATF_ERR_UNSUPPORTED
+    assert fasa(budget=4097) == atf.ATF_ERR_UNSUPPORTED
+    assert fasa(kv_len=[0]) == atf.ATF_ERR_INVALID_ARG
+    assert fasa(kv_len=[65]) == atf.ATF_ERR_INVALID_ARG
+    assert fasa(heads=36) == atf.ATF_ERR_UNSUPPORTED  # 9 query heads per kv head
+    assert fasa(heads=30) == atf.ATF_ERR_INVALID_ARG  # heads % kv_heads
+    assert fasa(d=96) == atf.ATF_ERR_UNSUPPORTED
+    assert fasa(wsb=fws - 1) == atf.ATF_ERR_INVALID_ARG and "workspace" in atf.atf_last_error()
+    assert fasa(ws=fake + 8) == atf.ATF_ERR_INVALID_ARG  # misaligned
+    assert fasa(ws=None) == atf.ATF_ERR_INVALID_ARG
     H = atf.atf_prefill_host
     need = atf.atf_prefill_host_workspace_bytes(1, 128, 128, 28, 4, 128, 0)
     assert _status(lambda: H(fake, fake, fake, fake, 1, 128, 128, 28, 4, 128, 0, 0, 1e7, 1.0, fake, need - 1)) == \
@@ -123,6 +145,7 @@ def test_empty_inputs_are_no_ops(lib):
     atf.atf_kv_append(None, None, None, None, 0, [], [], 8, 4, 128, 1e7)
     atf.atf_kv_append(None, None, None, None, 2, [0, 0], [3, 8], 8, 4, 128, 1e7)  # nothing to append
     atf.atf_prefill_host(None, None, None, None, 1, 0, 0, 28, 4, 128, 0, 0, 1e7, 1.0, None, 0)
+    atf.atf_fasa_decode(None, None, None, None, 0, [], 8, 28, 4, 128, 0xFF, 16)
 
 
 def test_workspace_sizes(lib):
@@ -135,6 +158,12 @@ def test_workspace_sizes(lib):
     assert hws == 3 * qb + 3 * kb
     assert atf.atf_prefill_host_workspace_bytes(2, 1000, 1500, 28, 4, 128, 1) == 2 * qb + 2 * kb
     assert atf.atf_prefill_host_workspace_bytes(0, 1000, 1500, 28, 4, 128, 0) == 0
+    # FASA: scores + candidates per (sequence, query head, key), 4096-bin histograms,
+    # two counters (padded to 256 bytes), the above-threshold and the selected
+    # indices, attention partials (128 selected keys per split)
+    fws = atf.atf_fasa_workspace_bytes(4, 28, 1 << 20, 2048, 128)
+    rows = 4 * 28
+    assert fws == rows * (1 << 20) * 8 + rows * 4096 * 4 + 1024 + 2 * rows * 2048 * 4 + rows * 16 * 130 * 4
     dws = atf.atf_decode_workspace_bytes(4, 28, 4, 1 << 20, 128)
     assert dws % (4 * 28 * 130 * 4) == 0 and dws > 0
 

@@ -1,0 +1,97 @@
+"""FASA-style decode (atf_fasa_decode) against the oracle: the scores and the
+selected key indices bit for bit, the output within the bf16 tolerance."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import fasa as ofasa
+from rope_frequency_sparse_b200 import atf, synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+LOW16 = 0xFFFF << 48  # the 16 lowest-frequency pairs of d = 128 (two cache chunks)
+
+
+def _inputs(B, N, Hq, Hkv, d, seed):
+    q = synth.token_major(seed, 901, 0, B, 1, Hq, d, torch.bfloat16, threads=1)[:, 0].contiguous()
+    k = synth.token_major(seed, 901, 1, B, N, Hkv, d, torch.bfloat16, threads=1)
+    v = synth.token_major(seed, 901, 2, B, N, Hkv, d, torch.bfloat16, threads=1)
+    return q, k, v
+
+
+def _chunked(k_rot):
+    """The chunk-major copy of already-rotated keys (a pure re-layout)."""
+    _, kc = atf.rope_layout(k_rot.cuda(), 1e4, rotate=False, rotated_out=False, chunked_out=True)
+    return kc
+
+
+def _run(q, k, v, kv_len, mask, budget):
+    B, Hq, d = q.shape
+    N = k.shape[1]
+    sel = torch.full((B, Hq, budget), -7, dtype=torch.int32, device="cuda")
+    sc = torch.full((B, Hq, N), float("nan"), dtype=torch.float32, device="cuda")
+    out = atf.fasa_decode(q.cuda(), _chunked(k), v.cuda(), kv_len, mask, budget, selected=sel, scores=sc)
+    atf.atf_check()
+    return out.cpu(), sel.cpu().numpy(), sc.cpu().numpy()
+
+
+def _check(q, k, v, kv_len, mask, budget):
+    out, sel, sc = _run(q, k, v, kv_len, mask, budget)
+    want, wsel, wsc = ofasa.fasa_decode(q, k, v, kv_len, mask, budget)
+    for b, L in enumerate(kv_len):
+        assert np.array_equal(sc[b, :, :L].view(np.uint32), wsc[b, :, :L].view(np.uint32)), b
+    assert np.array_equal(sel, wsel)
+    assert np.abs(out.double().numpy() - want).max() <= TOL
+    return sel
+
+
+@pytest.mark.parametrize("B,N,kv_len,Hq,Hkv,d,mask,budget", [
+    (2, 3000, [3000, 1337], 28, 4, 128, LOW16, 256),
+    (1, 5000, [4999], 7, 1, 128, (1 << 3) | (0xFF << 20) | (1 << 63), 1000),
+    (3, 700, [700, 1, 333], 4, 4, 64, 0b1010_0000_1111_0000_0000_0000_0000_0001, 100),
+    (1, 2048, [2048], 8, 1, 64, (1 << 32) - 1, 4096),  # budget above kv_len: every key
+])
+def test_fasa_matches_oracle(B, N, kv_len, Hq, Hkv, d, mask, budget):
+    q, k, v = _inputs(B, N, Hq, Hkv, d, seed=61)
+    _check(q, k, v, kv_len, mask, budget)
+
+
+def test_fasa_heavy_ties_use_every_radix_pass():
+    """Scores with five distinct values over 20000 keys: the budget boundary falls
+    inside a block of equal scores, decided by the key index alone."""
+    B, N, Hq, Hkv, d = 1, 20000, 2, 1, 64
+    g = np.random.default_rng(5)
+    q = torch.zeros(B, Hq, d)
+    q[:, :, 2 * 7] = 1.0
+    q[:, 1, 2 * 7] = -1.0
+    k = torch.zeros(B, N, Hkv, d)
+    k[..., 2 * 7] = torch.from_numpy(g.integers(-2, 3, size=(B, N, Hkv)).astype(np.float32))
+    v = torch.from_numpy(g.standard_normal((B, N, Hkv, d)).astype(np.float32))
+    q, k, v = q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+    sel = _check(q, k, v, [N], 1 << 7, 3001)
+    assert (sel >= 0).all()
+
+
+def test_fasa_without_optional_outputs_gives_the_same_result():
+    q, k, v = _inputs(2, 4096, 8, 2, 128, seed=67)
+    kv_len, budget = [4096, 2500], 300
+    out1, _, _ = _run(q, k, v, kv_len, LOW16, budget)
+    out2 = atf.fasa_decode(q.cuda(), _chunked(k), v.cuda(), kv_len, LOW16, budget).cpu()
+    atf.atf_check()
+    assert torch.equal(out1, out2)
+
+
+def test_fasa_full_size_cache():
+    """One sequence of the 4 x 2^20-token decode workload, 28 query heads, budget 2048."""
+    N, budget = 1 << 20, 2048
+    q = synth.token_major(71, 902, 0, 1, 1, 28, 128, torch.bfloat16, threads=4)[:, 0].contiguous()
+    k = synth.token_major(71, 902, 1, 1, N, 4, 128, torch.bfloat16, threads=4)
+    v = synth.token_major(71, 902, 2, 1, N, 4, 128, torch.bfloat16, threads=4)
+    out, sel, sc = _run(q, k, v, [N], LOW16, budget)
+    wsc = ofasa.tip_scores(q, k, [N], LOW16)
+    assert np.array_equal(sc.view(np.uint32), wsc.view(np.uint32))
+    wsel = ofasa.select(wsc, [N], budget)
+    assert np.array_equal(sel, wsel)
+    want = ofasa.focused_attention(q, k, v, wsel)
+    assert np.abs(out.double().numpy() - want).max() <= TOL
