@@ -479,6 +479,52 @@ def run_extra(args, device, stream, flush_buf, peaks):
                                      "traffic": recorded_traffic("decode.cu", "decode_1m.md")},
                         "data": "seeded torch CUDA normals (torch.Generator), bf16"}
 
+    # split-KV decode: the cache of every sequence split by key position across
+    # `world` ranks (traffic-balanced ranges), each rank's partial decode timed on
+    # its own copy of its range, plus the merge of the world partials
+    from rope_frequency_sparse_b200 import splitkv
+    skv = {}
+    part = torch.empty((w5.batch, w5.q_heads, w5.d + 2), dtype=torch.float32, device=device)
+    for world in (2, 4, 8):
+        ranges = splitkv.shard_ranges(N, world, w5.d, w5.theta, 1.0)
+        worst = 0.0
+        for r in (0, world - 1):  # the ranges farthest from and nearest to the query
+            lo, hi = ranges[r]
+            kc_r = kc[:, :, :, lo:hi, :].contiguous()
+            v_r = v5[:, lo:hi].contiguous()
+            need = atf.atf_decode_workspace_bytes(w5.batch, w5.q_heads, w5.kv_heads, hi - lo, w5.d)
+            ws_r = torch.empty(need, dtype=torch.uint8, device=device)
+
+            def prt(ev):
+                if ev:
+                    ev[0].record(stream)
+                atf.atf_decode_partial(q5, kc_r, v_r, part, w5.batch, [hi - lo] * w5.batch, [lo] * w5.batch,
+                                       [N - 1] * w5.batch, hi - lo, w5.q_heads, w5.kv_heads, w5.d, w5.theta, 1.0,
+                                       ws_r, need, None, s)
+                if ev:
+                    ev[1].record(stream)
+
+            evp = time_steps(prt, 10, 3, stream, flush_buf, n_events=2)
+            worst = max(worst, sum(e[0].elapsed_time(e[1]) for e in evp) / 10)
+            del kc_r, v_r, ws_r
+        parts = torch.zeros((world, w5.batch, w5.q_heads, w5.d + 2), dtype=torch.float32, device=device)
+
+        def mrg(ev):
+            if ev:
+                ev[0].record(stream)
+            atf.atf_decode_merge(parts, world, w5.batch, w5.q_heads, w5.d, o5, s)
+            if ev:
+                ev[1].record(stream)
+
+        evm = time_steps(mrg, 10, 3, stream, flush_buf, n_events=2)
+        ms_m = sum(e[0].elapsed_time(e[1]) for e in evm) / 10
+        skv[str(world)] = {"ms_rank_partial_max": worst, "ms_merge": ms_m,
+                           "speedup_vs_one_gpu_decode_excl_exchange": ms5 / (worst + ms_m),
+                           "exchange_bytes_per_rank": w5.batch * w5.q_heads * (w5.d + 2) * 4}
+    out["split_kv_decode_1m"] = dict(skv, note="per-rank partials timed one at a time on one GPU (the first and "
+                                               "last key ranges); the all-gather of the partials between GPUs is "
+                                               "not measured here")
+
     # FASA-style decode on the same cache: token scores on the 16 lowest-frequency
     # pairs (two 8-pair chunks), 2048 keys kept per query head, attention on those
     mask16, budget = 0xFFFF << 48, 2048

@@ -169,6 +169,34 @@ atf_status atf_decode(const void* q, const void* k_chunked, const void* v, void*
 /* Scratch bytes atf_decode needs for `batch` sequences of at most max_kv_len keys. */
 size_t atf_decode_workspace_bytes(int batch, int heads, int kv_heads, long long max_kv_len, int d);
 
+/* Decode over a key range, for a sequence whose cache is split across devices
+ * (each holds a contiguous range of positions) or otherwise into pieces.
+ * Sequence b's piece holds n_keys[b] rotated keys in slots 0 .. n_keys[b]-1, slot
+ * j at position key_pos0[b] + j; its query sits at position q_pos[b] (>= the last
+ * key's position) and is rotated there.  Windows and the causal order use those
+ * positions, so the pieces of a sequence give, merged, exactly atf_decode's
+ * softmax over all keys.
+ *   q, k_chunked, v, n_cache, heads, kv_heads, d, theta, alpha, pairing,
+ *   workspace, skipped_pairs: as in atf_decode (workspace sized with
+ *   atf_decode_workspace_bytes for the largest n_keys).
+ *   n_keys, key_pos0, q_pos: HOST arrays of batch entries; n_keys[b] may be 0 (an
+ *   empty piece merges as nothing).
+ *   partial: DEVICE fp32 [batch][heads][d + 2]: the piece's softmax numerator
+ *   (relative to its maximum), its maximum logit (log2 units, -inf when empty)
+ *   and its row sum: the form atf_decode_merge reads. */
+atf_status atf_decode_partial(const void* q, const void* k_chunked, const void* v, float* partial, int batch,
+                              const long long* n_keys, const long long* key_pos0, const long long* q_pos,
+                              long long n_cache, int heads, int kv_heads, int d, double theta, double alpha,
+                              int pairing, void* workspace, size_t workspace_bytes,
+                              unsigned long long* skipped_pairs, void* stream);
+
+/* Merges n_parts partials of atf_decode_partial, stored one after the other
+ * ([n_parts][batch][heads][d + 2] fp32, device), into out [batch][heads][d] bf16
+ * (log-sum-exp: each part's numerator and row sum are scaled by 2^(its max -
+ * the overall max)).  Parts whose maximum is -inf contribute nothing. */
+atf_status atf_decode_merge(const float* partials, int n_parts, int batch, int heads, int d, void* out,
+                            void* stream);
+
 /* Decode without any allocation: the same computation as atf_decode, but the
  * split-softmax partials live in a fixed 8 MiB device array inside the library
  * instead of a caller workspace.  The pages have no counterpart of this entry

@@ -68,6 +68,8 @@ def load_library(path: str = LIB_PATH):
         "atf_prefill_host": ([ctypes.POINTER(PrefillArgs), i, vp], i),
         "atf_decode": ([vp, vp, vp, vp, i, vp, ll, i, i, i, d, d, i, vp, sz, vp, vp], i),
         "atf_decode_workspace_bytes": ([i, i, i, ll, i], sz),
+        "atf_decode_partial": ([vp, vp, vp, vp, i, vp, vp, vp, ll, i, i, i, d, d, i, vp, sz, vp, vp], i),
+        "atf_decode_merge": ([vp, i, i, i, i, vp, vp], i),
         "atf_decode_noalloc": ([vp, vp, vp, vp, i, vp, ll, i, i, i, d, d, i, vp, vp], i),
         "atf_decode_noalloc_scratch_bytes": ([], sz),
         "atf_kv_append": ([vp, vp, vp, vp, i, vp, vp, ll, i, i, d, i, vp], i),
@@ -173,6 +175,23 @@ def atf_decode(q, k_chunked, v, out, batch, kv_len, n_cache, heads, kv_heads, d,
                                      kl.ctypes.data_as(ctypes.c_void_p), int(n_cache), heads, kv_heads, d,
                                      float(theta), float(alpha), int(pairing), _ptr(workspace),
                                      int(workspace_bytes), _ptr(skipped_pairs), _stream(stream)))
+
+
+def atf_decode_partial(q, k_chunked, v, partial, batch, n_keys, key_pos0, q_pos, n_cache, heads, kv_heads, d, theta,
+                       alpha, workspace, workspace_bytes, skipped_pairs=None, stream=None,
+                       pairing=ATF_PAIRS_INTERLEAVED):
+    """Decode over a key range (slots 0.. at positions key_pos0..; query at q_pos): the merged partial."""
+    arrs = [np.ascontiguousarray(np.asarray(x, dtype=np.int64).reshape(-1)) for x in (n_keys, key_pos0, q_pos)]
+    _check(load_library().atf_decode_partial(_ptr(q), _ptr(k_chunked), _ptr(v), _ptr(partial), batch,
+                                             *[a.ctypes.data_as(ctypes.c_void_p) for a in arrs], int(n_cache),
+                                             heads, kv_heads, d, float(theta), float(alpha), int(pairing),
+                                             _ptr(workspace), int(workspace_bytes), _ptr(skipped_pairs),
+                                             _stream(stream)))
+
+
+def atf_decode_merge(partials, n_parts, batch, heads, d, out, stream=None):
+    _check(load_library().atf_decode_merge(_ptr(partials), int(n_parts), batch, heads, d, _ptr(out),
+                                           _stream(stream)))
 
 
 def atf_decode_noalloc(q, k_chunked, v, out, batch, kv_len, n_cache, heads, kv_heads, d, theta, alpha,

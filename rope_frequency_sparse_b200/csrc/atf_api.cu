@@ -343,10 +343,19 @@ size_t atf_decode_workspace_bytes(int batch, int heads, int kv_heads, long long 
   return static_cast<size_t>(batch) * heads * ns * (d + 2) * sizeof(float);
 }
 
-atf_status atf_decode(const void* q, const void* k_chunked, const void* v, void* out, int batch,
-                      const long long* kv_len, long long n_cache, int heads, int kv_heads, int d, double theta,
-                      double alpha, int pairing, void* workspace, size_t workspace_bytes,
-                      unsigned long long* skipped_pairs, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The decode of atf_decode and atf_decode_partial.  Sequence b's cache holds
+// n_keys[b] keys in slots 0.., slot 0 at position key_pos0[b] (0 when NULL); its
+// query sits at q_pos[b] (n_keys[b] - 1 + key_pos0[b] when NULL).  Writes the
+// bf16 output, or with partial_out the merged partial of these keys.
+atf_status decode_impl(const void* q, const void* k_chunked, const void* v, void* out, float* partial_out,
+                       int batch, const long long* n_keys, const long long* key_pos0, const long long* q_pos,
+                       long long n_cache, int heads, int kv_heads, int d, double theta, double alpha, int pairing,
+                       void* workspace, size_t workspace_bytes, unsigned long long* skipped_pairs, void* stream) {
+  const bool partial = partial_out != nullptr;
   if (atf_status st = check_params(d, theta, alpha)) return st;
   if (pairing != ATF_PAIRS_INTERLEAVED && pairing != ATF_PAIRS_ROTATE_HALF)
     return fail(ATF_ERR_INVALID_ARG, "decode: pairing %d", pairing);
@@ -355,14 +364,21 @@ atf_status atf_decode(const void* q, const void* k_chunked, const void* v, void*
   if (heads / kv_heads > 8) return fail(ATF_ERR_UNSUPPORTED, "decode: at most 8 query heads per kv head");
   if (n_cache > 0x7fffffffLL) return fail(ATF_ERR_UNSUPPORTED, "decode: cache longer than 2^31-1");
   if (batch == 0) return ATF_OK;
-  if (!q || !k_chunked || !v || !out || !kv_len) return fail(ATF_ERR_INVALID_ARG, "decode: null pointer");
-  if (!aligned16(q) || !aligned16(k_chunked) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
+  if (!q || !k_chunked || !v || !(out || partial_out) || !n_keys) return fail(ATF_ERR_INVALID_ARG, "decode: null pointer");
+  if (!aligned16(q) || !aligned16(k_chunked) || !aligned16(v) || (out && !aligned16(out)) ||
+      (partial_out && !aligned16(partial_out)) || !aligned16(workspace))
     return fail(ATF_ERR_INVALID_ARG, "decode: pointers must be 16-byte aligned");
   long long max_len = 0;
   for (int b = 0; b < batch; ++b) {
-    if (kv_len[b] < 1 || kv_len[b] > n_cache)
-      return fail(ATF_ERR_INVALID_ARG, "decode: kv_len[%d]=%lld outside [1, n_cache]", b, kv_len[b]);
-    if (kv_len[b] > max_len) max_len = kv_len[b];
+    const long long lo = partial ? 0 : 1;  // a key range may be empty; a whole sequence holds its query's key
+    if (n_keys[b] < lo || n_keys[b] > n_cache)
+      return fail(ATF_ERR_INVALID_ARG, "decode: kv_len[%d]=%lld outside [%lld, n_cache]", b, n_keys[b], lo);
+    const long long p0 = key_pos0 ? key_pos0[b] : 0;
+    const long long qp = q_pos ? q_pos[b] : p0 + n_keys[b] - 1;
+    if (p0 < 0 || qp < 0 || qp < p0 + n_keys[b] - 1 || qp > (1LL << 40))
+      return fail(ATF_ERR_INVALID_ARG, "decode: sequence %d: the query (position %lld) must not precede its keys "
+                  "(positions %lld ..%lld)", b, qp, p0, p0 + n_keys[b] - 1);
+    if (n_keys[b] > max_len) max_len = n_keys[b];
   }
   const size_t need = atf_decode_workspace_bytes(batch, heads, kv_heads, max_len, d);
   if (!workspace || workspace_bytes < need)
@@ -389,11 +405,16 @@ atf_status atf_decode(const void* q, const void* k_chunked, const void* v, void*
   for (int b0 = 0; b0 < batch; b0 += kMaxDecodeBatch) {
     const int nb = batch - b0 < kMaxDecodeBatch ? batch - b0 : kMaxDecodeBatch;
     p.batch = nb;
-    for (int i = 0; i < nb; ++i) p.kv_len[i] = kv_len[b0 + i];
+    for (int i = 0; i < nb; ++i) {
+      p.kv_len[i] = n_keys[b0 + i];
+      p.key_pos0[i] = key_pos0 ? key_pos0[b0 + i] : 0;
+      p.q_pos[i] = q_pos ? q_pos[b0 + i] : p.key_pos0[i] + p.kv_len[i] - 1;
+    }
     p.q = static_cast<const char*>(q) + static_cast<size_t>(b0) * heads * d * esz;
     p.kc = static_cast<const char*>(k_chunked) + static_cast<size_t>(b0) * kv_heads * n_cache * d * esz;
     p.v = static_cast<const char*>(v) + static_cast<size_t>(b0) * n_cache * kv_heads * d * esz;
-    p.out = static_cast<char*>(out) + static_cast<size_t>(b0) * heads * d * esz;
+    p.out = out ? static_cast<char*>(out) + static_cast<size_t>(b0) * heads * d * esz : nullptr;
+    p.partial_out = partial_out ? partial_out + static_cast<size_t>(b0) * heads * (d + 2) : nullptr;
     p.partials = static_cast<float*>(workspace) + static_cast<size_t>(b0) * heads * ns * (d + 2);
     CUtensorMap tv, tk;
     if (atf_status st = kv_tensor_map(&tv, p.v, nb, static_cast<int>(n_cache), kv_heads, d)) return st;
@@ -401,6 +422,43 @@ atf_status atf_decode(const void* q, const void* k_chunked, const void* v, void*
     cudaError_t e = launch_decode(p, tv, tk, s);
     if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
   }
+  return ATF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+atf_status atf_decode(const void* q, const void* k_chunked, const void* v, void* out, int batch,
+                      const long long* kv_len, long long n_cache, int heads, int kv_heads, int d, double theta,
+                      double alpha, int pairing, void* workspace, size_t workspace_bytes,
+                      unsigned long long* skipped_pairs, void* stream) {
+  if (batch > 0 && !out) return fail(ATF_ERR_INVALID_ARG, "decode: null pointer");
+  return decode_impl(q, k_chunked, v, out, nullptr, batch, kv_len, nullptr, nullptr, n_cache, heads, kv_heads, d,
+                     theta, alpha, pairing, workspace, workspace_bytes, skipped_pairs, stream);
+}
+
+atf_status atf_decode_partial(const void* q, const void* k_chunked, const void* v, float* partial, int batch,
+                              const long long* n_keys, const long long* key_pos0, const long long* q_pos,
+                              long long n_cache, int heads, int kv_heads, int d, double theta, double alpha,
+                              int pairing, void* workspace, size_t workspace_bytes,
+                              unsigned long long* skipped_pairs, void* stream) {
+  if (batch > 0 && (!partial || !key_pos0 || !q_pos)) return fail(ATF_ERR_INVALID_ARG, "decode_partial: null pointer");
+  return decode_impl(q, k_chunked, v, nullptr, partial, batch, n_keys, key_pos0, q_pos, n_cache, heads, kv_heads, d,
+                     theta, alpha, pairing, workspace, workspace_bytes, skipped_pairs, stream);
+}
+
+atf_status atf_decode_merge(const float* partials, int n_parts, int batch, int heads, int d, void* out,
+                            void* stream) {
+  if (d != 64 && d != 128) return fail(ATF_ERR_UNSUPPORTED, "head dim d=%d not supported (64 or 128)", d);
+  if (n_parts < 1 || batch < 0 || heads < 1) return fail(ATF_ERR_INVALID_ARG, "decode_merge: bad sizes");
+  if (batch == 0) return ATF_OK;
+  if (!partials || !out) return fail(ATF_ERR_INVALID_ARG, "decode_merge: null pointer");
+  if (!aligned16(partials) || !aligned16(out))
+    return fail(ATF_ERR_INVALID_ARG, "decode_merge: pointers must be 16-byte aligned");
+  cudaError_t e = launch_decode_merge(partials, n_parts, static_cast<long long>(batch) * heads, d, out,
+                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode merge launch");
   return ATF_OK;
 }
 

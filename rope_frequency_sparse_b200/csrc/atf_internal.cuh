@@ -50,7 +50,10 @@ struct DecodeParams {
   int batch, hq, hkv, d, n_split;
   int pairing;           // atf_pairing of the raw queries
   long long n_cache;
-  long long kv_len[kMaxDecodeBatch];
+  long long kv_len[kMaxDecodeBatch];    // keys in this cache: slots 0 .. kv_len-1
+  long long q_pos[kMaxDecodeBatch];     // query position (its RoPE angle)
+  long long key_pos0[kMaxDecodeBatch];  // position of slot 0 (a key range of a longer sequence)
+  float* partial_out;           // nullable: [B][Hq][d + 2] merged (sum, max, row sum) instead of out
   unsigned long long* skipped;  // nullable
   unsigned int* err;
   Windows win;
@@ -75,6 +78,7 @@ cudaError_t launch_kv_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillParams& p, cudaStream_t s);
 cudaError_t launch_prefill_tc(const PrefillParams& p, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                               const CUtensorMap& tm_v, bool dense, cudaStream_t s);
+cudaError_t launch_decode_merge(const float* parts, int n_parts, long long rows, int d, void* out, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tm_v, const CUtensorMap& tm_k,
                           cudaStream_t s);
 

@@ -80,18 +80,20 @@ __device__ long long traffic_below(long long x, const int* sW, int nc) {
   return t;
 }
 
-// First key index of split s (of ns) over keys [0, L), the query at L-1.
-__device__ long long split_begin(int s, int ns, long long L, const int* sW, int nc) {
+// First key index of split s (of ns) over keys [0, L) whose key 0 lies at
+// distance q1 - 1 from the query (q1 = L for a whole sequence, the query at L-1).
+// Keys [0, n) have distances [q1 - n, q1), hence traffic T(q1) - T(q1 - n).
+__device__ long long split_begin(int s, int ns, long long L, long long q1, const int* sW, int nc) {
   if (s <= 0) return 0;
   if (s >= ns) return L;
-  const long long total = traffic_below(L, sW, nc);
-  // keys [0, n) have traffic total - traffic_below(L - n); find the smallest n
-  // with that >= s*total/ns.
+  const long long top = traffic_below(q1, sW, nc);
+  const long long total = top - traffic_below(q1 - L, sW, nc);
+  // the smallest n with traffic of keys [0, n) >= s*total/ns
   const long long target = (total / ns) * s + ((total % ns) * s) / ns;
   long long lo = 0, hi = L;
   while (lo < hi) {
     const long long mid = (lo + hi) / 2;
-    if (total - traffic_below(L - mid, sW, nc) >= target)
+    if (top - traffic_below(q1 - mid, sW, nc) >= target)
       hi = mid;
     else
       lo = mid + 1;
@@ -132,7 +134,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const long long L = p.kv_len[b];
-  const long long qpos = L - 1;
+  const long long qpos = p.q_pos[b];              // RoPE angle of the query
+  const long long qloc = qpos - p.key_pos0[b];    // the query's distance from slot 0
 
   if (tid == 0) {
     for (int s = 0; s < NSTG; ++s) {
@@ -167,13 +170,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
   __syncthreads();
 
-  const long long nb = split_begin(split, p.n_split, L, sh->w, NC);
-  const long long ne = split_begin(split + 1, p.n_split, L, sh->w, NC);
+  const long long nb = split_begin(split, p.n_split, L, qloc + 1, sh->w, NC);
+  const long long ne = split_begin(split + 1, p.n_split, L, qloc + 1, sh->w, NC);
   const int ntiles = ne > nb ? static_cast<int>((ne - nb + BKD - 1) / BKD) : 0;
   volatile int* abort = &sh->abort;
   auto tile_dead_chunks = [&](int t) {
     const long long last = min(nb + static_cast<long long>(t) * BKD + BKD - 1, ne - 1);
-    return dead_chunks(sh->w, NC, qpos - last);
+    return dead_chunks(sh->w, NC, qloc - last);
   };
 
   // per-warp softmax state (consumers): row hrow = lane / 4 of the accumulators
@@ -238,7 +241,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       // distance of this lane's B column key in each of the warp's four 8-key n-tiles
       long long dl[4];
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) dl[nt] = qpos - (n0 + 32 * w + 8 * nt + (lane >> 2));
+      for (int nt = 0; nt < 4; ++nt) dl[nt] = qloc - (n0 + 32 * w + 8 * nt + (lane >> 2));
 
       // ---- S = Q~ K~^T over the live chunks, B registers zeroed for pairs outside their window
       float sfr[4][4];
@@ -325,7 +328,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           for (int c = 0; c < NC; ++c) dead += (dl[nt] > wlo[c]) + (dl[nt] > whi[c]);
           dead += __shfl_xor_sync(0xffffffffu, dead, 1);
           dead += __shfl_xor_sync(0xffffffffu, dead, 2);
-          if ((lane & 3) == 0 && qpos - dl[nt] < ne) cnt += static_cast<unsigned long long>(dead) * G;
+          if ((lane & 3) == 0 && qloc - dl[nt] < ne) cnt += static_cast<unsigned long long>(dead) * G;
         }
       }
     }
@@ -394,8 +397,37 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeParams p) {
     a += part[s * (D + 2) + e] * f;
     l += part[s * (D + 2) + D + 1] * f;
   }
+  if (p.partial_out) {  // this key range's merged partial, for a merge with other ranges
+    float* pp = p.partial_out + (static_cast<long long>(b) * p.hq + h) * (D + 2);
+    pp[e] = a;
+    if (e == 0) {
+      pp[D] = M;
+      pp[D + 1] = l;
+    }
+    return;
+  }
   __nv_bfloat16* O = static_cast<__nv_bfloat16*>(p.out) + (static_cast<long long>(b) * p.hq + h) * D;
   O[e] = __float2bfloat16(l > 0.f ? a / l : 0.f);
+}
+
+// Merge n_parts partials [n_parts][rows][D + 2] (sum relative to the max, max in
+// log2 units, row sum) into the bf16 output [rows][D].
+template <int D>
+__global__ void __launch_bounds__(D) decode_merge_kernel(const float* parts, int n_parts, long long rows,
+                                                         __nv_bfloat16* out) {
+  const long long row = blockIdx.x;
+  const int e = threadIdx.x;
+  float M = -INFINITY;
+  for (int r = 0; r < n_parts; ++r) M = fmaxf(M, parts[(r * rows + row) * (D + 2) + D]);
+  float a = 0.f, l = 0.f;
+  for (int r = 0; r < n_parts; ++r) {
+    const float* pr = parts + (r * rows + row) * (D + 2);
+    if (pr[D] == -INFINITY) continue;
+    const float f = ex2_approx(pr[D] - M);
+    a += pr[e] * f;
+    l += pr[D + 1] * f;
+  }
+  out[row * D + e] = __float2bfloat16(l > 0.f ? a / l : 0.f);
 }
 
 int decode_num_splits(long long max_kv_len, int batch, int hkv) {
@@ -445,6 +477,16 @@ static cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap& tv,
   }
   if (e != cudaSuccess) return e;
   decode_combine_kernel<D><<<dim3(p.hq, p.batch), D, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_merge(const float* parts, int n_parts, long long rows, int d, void* out, cudaStream_t s) {
+  if (rows == 0) return cudaSuccess;
+  auto* o = static_cast<__nv_bfloat16*>(out);
+  if (d == 64)
+    decode_merge_kernel<64><<<static_cast<unsigned>(rows), 64, 0, s>>>(parts, n_parts, rows, o);
+  else
+    decode_merge_kernel<128><<<static_cast<unsigned>(rows), 128, 0, s>>>(parts, n_parts, rows, o);
   return cudaGetLastError();
 }
 

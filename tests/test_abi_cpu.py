@@ -92,6 +92,16 @@ def test_rejects_bad_arguments_before_any_device_call(lib):
     assert _status(lambda: A(fake + 8, fake, fake, fake, 1, [1], [0], 8, 4, 128, 1e7)) == \
         atf.ATF_ERR_INVALID_ARG  # misaligned
     assert _status(lambda: A(fake, fake, fake, fake, 1, [1], [0], 8, 4, 96, 1e7)) == atf.ATF_ERR_UNSUPPORTED
+    DP = atf.atf_decode_partial
+    assert _status(lambda: DP(fake, fake, fake, fake, 1, [5], [10], [13], 8, 28, 4, 128, 1e7, 1.0, fake,
+                              1 << 20)) == atf.ATF_ERR_INVALID_ARG  # query before the last key (14)
+    assert _status(lambda: DP(fake, fake, fake, fake, 1, [9], [0], [100], 8, 28, 4, 128, 1e7, 1.0, fake,
+                              1 << 20)) == atf.ATF_ERR_INVALID_ARG  # more keys than slots
+    assert _status(lambda: DP(fake, fake, fake, fake, 1, [2], [-1], [100], 8, 28, 4, 128, 1e7, 1.0, fake,
+                              1 << 20)) == atf.ATF_ERR_INVALID_ARG  # negative position
+    assert _status(lambda: atf.atf_decode_merge(fake, 0, 1, 28, 128, fake)) == atf.ATF_ERR_INVALID_ARG
+    assert _status(lambda: atf.atf_decode_merge(fake, 2, 1, 28, 96, fake)) == atf.ATF_ERR_UNSUPPORTED
+    assert _status(lambda: atf.atf_decode_merge(fake + 4, 2, 1, 28, 128, fake)) == atf.ATF_ERR_INVALID_ARG
     F = atf.atf_fasa_decode
     fws = atf.atf_fasa_workspace_bytes(1, 28, 64, 16, 128)
     ok_args = dict(batch=1, kv_len=[64], n_cache=64, heads=28, kv_heads=4, d=128, pair_mask=0xFF, budget=16)
