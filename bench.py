@@ -614,6 +614,36 @@ def run_decode_profile(args):
                       "ms_per_step": e0.elapsed_time(e1) / max(args.steps, 1)}))
 
 
+def run_fasa_profile(args):
+    """Only the FASA-style decode with a shortened cache, for ncu captures: one
+    sequence of KEYS cached keys, 28/4 heads, d = 128, the 16 lowest-frequency
+    pairs dominant, 2048 keys kept per query head; W + K calls."""
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    w5 = synth.WORKLOADS["decode_1m"]
+    N, B = args.profile_fasa, 1
+    g = torch.Generator(device=device)
+    g.manual_seed(synth.DEFAULT_SEED)
+    kc = torch.randn((B, w5.kv_heads, w5.d // 16, N, 16), generator=g, device=device).to(torch.bfloat16)
+    v5 = torch.randn((B, N, w5.kv_heads, w5.d), generator=g, device=device).to(torch.bfloat16)
+    q5 = torch.randn((B, w5.q_heads, w5.d), generator=g, device=device).to(torch.bfloat16)
+    o5 = torch.empty_like(q5)
+    budget = 2048
+    ws_b = atf.atf_fasa_workspace_bytes(B, w5.q_heads, N, budget, w5.d)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device=device)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for it in range(args.warmup + args.steps):
+        if it == args.warmup:
+            e0.record(s)
+        atf.atf_fasa_decode(q5, kc, v5, o5, B, [N], N, w5.q_heads, w5.kv_heads, w5.d, 0xFFFF << 48, budget, None,
+                            None, ws, ws_b, s)
+    e1.record(s)
+    atf.atf_check(s)
+    print(json.dumps({"profile": "fasa", "keys": N, "batch": B, "calls": args.warmup + args.steps,
+                      "ms_per_call": e0.elapsed_time(e1) / max(args.steps, 1)}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -624,10 +654,15 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--profile-decode", type=int, metavar="KEYS", default=0,
                     help="run only the decode step with KEYS cached keys per sequence (for ncu captures)")
+    ap.add_argument("--profile-fasa", type=int, metavar="KEYS", default=0,
+                    help="run only the FASA-style decode on one sequence of KEYS keys (for ncu captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.profile_decode:
         run_decode_profile(args)
+        return
+    if args.profile_fasa:
+        run_fasa_profile(args)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

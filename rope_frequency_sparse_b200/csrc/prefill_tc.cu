@@ -459,14 +459,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         int cmax = -1;
         if (row_ok) cmax = static_cast<int>(min(static_cast<long long>(BN - 1), min(m, kv_last) - n0));
         const bool partial = __any_sync(0xffffffffu, cmax < BN - 1);
-        if (!(ok = warp_wait(&sh->s_full[g], (j - j0) & 1, abort, p.err, 0x303))) break;
-        tc_fence_after();
+        // (everything up to the wait is independent of S, off the softmax -> MMA chain)
         // no S MMA when every pair is zeroed in every row
         const bool has_mma = !SPARSE || (ww.below(center + kZeroOffset) >> 3) < C::NCH;
+        const int nv = cmax + 1;  // valid columns of this row
+        if (SPARSE) cnt += static_cast<unsigned long long>(a) * nv;
+        const int cmax_w = (SPARSE && a < u) ? __reduce_max_sync(0xffffffffu, cmax) : 0;
+        if (!(ok = warp_wait(&sh->s_full[g], (j - j0) & 1, abort, p.err, 0x303))) break;
+        tc_fence_after();
         uint32_t s_chunks = has_mma ? 0xFu : 0u;  // 32-column chunks of S held in TMEM
         if (SPARSE) {
-          const int nv = cmax + 1;  // valid columns of this row
-          cnt += static_cast<unsigned long long>(a) * nv;
           if (__builtin_expect(a < u, 0)) {
             // ---- boundary corrections, in place on S in TMEM, 32 columns at a time.
             // For pairs in [a, u) the windows lie within 127 of the centre, so the
@@ -477,8 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t q_base = smem_u32(sQg);
             const uint32_t stash_base = smem_u32(&sh->stash[g][0][r]);
             // chunks past every row's last valid column (beyond the causal diagonal
-            // or the last key) are masked out whole: nothing there needs correcting
-            const int cmax_w = __reduce_max_sync(0xffffffffu, cmax);
+            // or the last key, cmax_w) are masked out whole: nothing there needs correcting
 #pragma unroll 1
             for (int hb = a; hb < u; hb += 32) {
               // classify pair hb + lane: the chunks some row of this warp must
