@@ -16,9 +16,9 @@
 //      scores go to memory, with a 4096-bin histogram per query head of the top
 //      12 bits of their order-preserving bit pattern (sign, exponent and three
 //      mantissa bits: a bin spans an eighth of an octave).
-//   2. fasa_scan_kernel: 32 CTAs per (query head, sequence).  From the
-//      histogram each finds the bin holding the budget-th largest score, then
-//      sweeps its 1/32 of the scores: keys above that bin are in (appended to
+//   2. fasa_threshold_kernel (one CTA per row) finds from the histogram the bin
+//      holding the budget-th largest score; fasa_scan_kernel, 32 CTAs per
+//      (query head, sequence), then sweeps 1/32 of the scores each: keys above that bin are in (appended to
 //      an unsorted list), keys in it are candidates.
 //   3. fasa_finish_kernel: one CTA per (query head, sequence).  Radix passes over
 //      the candidates on the rest of the 64-bit selection key (score bits, then
@@ -66,6 +66,7 @@ struct FasaParams {
   uint32_t* cand;           // [B][Hq][n_cache] candidates of the threshold bin
   unsigned int* hist;       // [B][Hq][kHistBins]
   unsigned int* counts;     // [B][Hq][2]: keys above the threshold bin, candidates
+  int* thr;                 // [B][Hq]: the threshold bin
   int* above;               // [B][Hq][budget]: keys above the threshold bin, unsorted
   int* sel;                 // [B][Hq][budget], ascending, -1 padded
   float* partials;          // [B][Hq][n_split][d + 2]
@@ -81,24 +82,22 @@ __device__ __forceinline__ uint32_t order_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kScoreThreads) fasa_score_kernel(FasaParams p) {
+template <int D, int G>
+__global__ void __launch_bounds__(kScoreThreads, 3) fasa_score_kernel(FasaParams p) {  // 3 CTAs per SM
   constexpr int NC = D / 16;
   const int kvh = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-  const int G = p.hq / p.hkv;
   const long long L = p.kv_len[b];
   const long long n0 = static_cast<long long>(blockIdx.x) * kScoreKeys;
   if (n0 >= L) return;
-  __shared__ uint4 sq[kMaxG][D / 2];  // (q_2i, q_2i, q_2i+1, q_2i+1) per head and pair
+  __shared__ ulonglong2 sq[G][D / 2];  // ((q_2i, q_2i), (q_2i+1, q_2i+1)) per head and pair, as f32x2
   // per head, kHistBins 16-bit counts packed two to a word (a CTA scores at most
   // kScoreKeys < 2^16 keys)
   extern __shared__ unsigned int shist[];
   for (int i = tid; i < G * (D / 2); i += kScoreThreads) {
     const int g = i / (D / 2), pr = i % (D / 2);
     const __nv_bfloat16* qh = p.q + (static_cast<long long>(b) * p.hq + kvh * G + g) * D;
-    const uint32_t qa = __float_as_uint(__bfloat162float(qh[2 * pr]));
-    const uint32_t qb = __float_as_uint(__bfloat162float(qh[2 * pr + 1]));
-    sq[g][pr] = make_uint4(qa, qa, qb, qb);
+    const float qa = __bfloat162float(qh[2 * pr]), qb = __bfloat162float(qh[2 * pr + 1]);
+    sq[g][pr] = make_ulonglong2(pack2(qa, qa), pack2(qb, qb));
   }
   for (int i = tid; i < G * (kHistBins / 2); i += kScoreThreads) shist[i] = 0u;
   __syncthreads();
@@ -121,9 +120,9 @@ __global__ void __launch_bounds__(kScoreThreads) fasa_score_kernel(FasaParams p)
       vk[k] = nk[k] < L;
     }
     if (!vk[0]) break;
-    uint64_t s2[2][kMaxG];
+    uint64_t s2[2][G];
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g) s2[0][g] = s2[1][g] = 0ull;  // (+0, +0)
+    for (int g = 0; g < G; ++g) s2[0][g] = s2[1][g] = 0ull;  // (+0, +0)
 #pragma unroll 1
     for (int c = 0; c < NC; ++c) {
       const uint32_t bits = static_cast<uint32_t>((p.mask >> (8 * c)) & 0xFFu);
@@ -149,23 +148,19 @@ __global__ void __launch_bounds__(kScoreThreads) fasa_score_kernel(FasaParams p)
           k1[h2] = pack2(__uint_as_float(w0 & 0xFFFF0000u), __uint_as_float(w1 & 0xFFFF0000u));
         }
 #pragma unroll
-        for (int g = 0; g < kMaxG; ++g) {
-          if (g < G) {
-            const uint4 qp = sq[g][8 * c + j];
-            const uint64_t qa = (static_cast<uint64_t>(qp.y) << 32) | qp.x;
-            const uint64_t qb = (static_cast<uint64_t>(qp.w) << 32) | qp.z;
+        for (int g = 0; g < G; ++g) {
+          const ulonglong2 qp = sq[g][8 * c + j];
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              s2[h2][g] = ffma2(qa, k0[h2], s2[h2][g]);  // dim 2i
-              s2[h2][g] = ffma2(qb, k1[h2], s2[h2][g]);  // dim 2i+1
-            }
+          for (int h2 = 0; h2 < 2; ++h2) {
+            s2[h2][g] = ffma2(qp.x, k0[h2], s2[h2][g]);  // dim 2i
+            s2[h2][g] = ffma2(qp.y, k1[h2], s2[h2][g]);  // dim 2i+1
           }
         }
       }
     }
 #pragma unroll
-    for (int g = 0; g < kMaxG; ++g) {
-      if (g < G) {
+    for (int g = 0; g < G; ++g) {
+      {
         float* srow = p.scores + (static_cast<long long>(b) * p.hq + kvh * G + g) * p.n_cache;
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -239,22 +234,27 @@ __device__ __forceinline__ void warp_append(bool flag, uint32_t value, unsigned 
   if (flag && slot < capacity) list[slot] = value;
 }
 
-__global__ void __launch_bounds__(kScanThreads) fasa_scan_kernel(FasaParams p) {
-  const int part = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+// The threshold bin of every (query head, sequence) row: the histogram bin holding
+// the need-th largest score (kHistBins when every key is selected: nothing to
+// sweep).  Thread t holds the 16 bins [4096 - 16 (t + 1), 4096 - 16 t), scanned
+// from the top.
+__global__ void __launch_bounds__(kScanThreads) fasa_threshold_kernel(FasaParams p) {
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const long long row = static_cast<long long>(b) * p.hq + h;
   const int L = static_cast<int>(p.kv_len[b]);
   const int need = L < p.budget ? L : p.budget;
-  if (need == L) return;  // every key is selected; the finishing kernel lists them
   __shared__ int s_scan[kScanThreads];
-  __shared__ int s_thr;
-  // The threshold bin: the bin holding the need-th largest score.  Thread t holds
-  // the 16 bins [4096 - 16 (t + 1), 4096 - 16 t), scanned from the top.
+  if (need == L) {
+    if (tid == 0) p.thr[row] = kHistBins;
+    return;
+  }
   constexpr int kPer = kHistBins / kScanThreads;
   const unsigned int* hg = p.hist + row * kHistBins;
   int mine = 0;
 #pragma unroll
   for (int k = 0; k < kPer; ++k) mine += static_cast<int>(hg[kHistBins - kPer * tid - 1 - k]);
   s_scan[tid] = mine;
+  if (tid == 0) p.thr[row] = kHistBins;  // no bin (emits nothing) unless the search below finds one
   __syncthreads();
   for (int off = 1; off < kScanThreads; off <<= 1) {  // inclusive scan (Hillis-Steele)
     const int t = tid >= off ? s_scan[tid - off] : 0;
@@ -262,8 +262,6 @@ __global__ void __launch_bounds__(kScanThreads) fasa_scan_kernel(FasaParams p) {
     s_scan[tid] += t;
     __syncthreads();
   }
-  if (tid == 0) s_thr = kHistBins;  // no bin (emits nothing) unless the search below finds one
-  __syncthreads();
   const int incl = s_scan[tid], excl = incl - mine;
   if (excl < need && need <= incl) {
     int acc = excl;
@@ -271,13 +269,19 @@ __global__ void __launch_bounds__(kScanThreads) fasa_scan_kernel(FasaParams p) {
       const int bin = kHistBins - kPer * tid - 1 - k;
       acc += static_cast<int>(hg[bin]);
       if (acc >= need) {
-        s_thr = bin;
+        p.thr[row] = bin;
         break;
       }
     }
   }
-  __syncthreads();
-  const uint32_t thr = static_cast<uint32_t>(s_thr);
+}
+
+__global__ void __launch_bounds__(kScanThreads) fasa_scan_kernel(FasaParams p) {
+  const int part = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const long long row = static_cast<long long>(b) * p.hq + h;
+  const int L = static_cast<int>(p.kv_len[b]);
+  const uint32_t thr = static_cast<uint32_t>(p.thr[row]);
+  if (thr >= static_cast<uint32_t>(kHistBins)) return;  // every key is selected (or nothing to find)
   // this CTA's share of the keys (a multiple of 4 long, so that rows of a cache
   // whose length is a multiple of 4 are read as float4)
   const int per = ((L + kScanCtas - 1) / kScanCtas + 3) & ~3;
@@ -301,6 +305,17 @@ __global__ void __launch_bounds__(kScanThreads) fasa_scan_kernel(FasaParams p) {
         const int idx = base + 4 * (u * kScanThreads + tid);
         v[u] = idx < n_hi ? __ldg(reinterpret_cast<const float4*>(sc + idx)) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
+      // almost every score lies below the threshold bin: one vote per warp skips
+      // the appends unless some lane holds a key at or above it
+      bool hit = false;
+#pragma unroll
+      for (int u = 0; u < kScanUnroll4; ++u) {
+        const int idx = base + 4 * (u * kScanThreads + tid);
+        if (idx < n_hi)
+          hit |= max(max(order_key(v[u].x), order_key(v[u].y)), max(order_key(v[u].z), order_key(v[u].w))) >>
+                     (32 - kHistBits) >= thr;
+      }
+      if (!__any_sync(0xffffffffu, hit)) continue;
 #pragma unroll
       for (int u = 0; u < kScanUnroll4; ++u) {
         const int idx = base + 4 * (u * kScanThreads + tid);
@@ -560,7 +575,7 @@ __global__ void __launch_bounds__(D) fasa_combine_kernel(FasaParams p) {
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct FasaLayout {
-  size_t scores, cand, hist, counts, above, sel, partials, total;
+  size_t scores, cand, hist, counts, thr, above, sel, partials, total;
 };
 
 FasaLayout fasa_layout(int batch, int heads, long long n_cache, int budget, int d, bool own_scores, bool own_sel) {
@@ -576,6 +591,8 @@ FasaLayout fasa_layout(int batch, int heads, long long n_cache, int budget, int 
   off += rows * kHistBins * sizeof(unsigned int);
   L.counts = off;
   off += align256(rows * 2 * sizeof(unsigned int));
+  L.thr = off;
+  off += align256(rows * sizeof(int));
   L.above = off;
   off += align256(rows * budget * sizeof(int));
   L.sel = off;
@@ -595,13 +612,34 @@ cudaError_t launch_fasa(const FasaParams& p, long long max_len, cudaStream_t s) 
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !(configured & (1ull << dev))) {
-    e = cudaFuncSetAttribute(fasa_score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kMaxG * (kHistBins / 2) * static_cast<int>(sizeof(unsigned int)));
-    if (e != cudaSuccess) return e;
+    const int bytes = kMaxG * (kHistBins / 2) * static_cast<int>(sizeof(unsigned int));
+    const void* fns[8] = {reinterpret_cast<const void*>(fasa_score_kernel<D, 1>),
+                          reinterpret_cast<const void*>(fasa_score_kernel<D, 2>),
+                          reinterpret_cast<const void*>(fasa_score_kernel<D, 3>),
+                          reinterpret_cast<const void*>(fasa_score_kernel<D, 4>),
+                          reinterpret_cast<const void*>(fasa_score_kernel<D, 5>),
+                          reinterpret_cast<const void*>(fasa_score_kernel<D, 6>),
+                          reinterpret_cast<const void*>(fasa_score_kernel<D, 7>),
+                          reinterpret_cast<const void*>(fasa_score_kernel<D, 8>)};
+    for (const void* f : fns) {
+      e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+      if (e != cudaSuccess) return e;
+    }
     if (dev < 64) configured |= 1ull << dev;
   }
   const unsigned nblk = static_cast<unsigned>((max_len + kScoreKeys - 1) / kScoreKeys);
-  fasa_score_kernel<D><<<dim3(nblk, p.hkv, p.batch), kScoreThreads, hist_smem, s>>>(p);
+  const dim3 grid(nblk, p.hkv, p.batch);
+  switch (G) {
+    case 1: fasa_score_kernel<D, 1><<<grid, kScoreThreads, hist_smem, s>>>(p); break;
+    case 2: fasa_score_kernel<D, 2><<<grid, kScoreThreads, hist_smem, s>>>(p); break;
+    case 3: fasa_score_kernel<D, 3><<<grid, kScoreThreads, hist_smem, s>>>(p); break;
+    case 4: fasa_score_kernel<D, 4><<<grid, kScoreThreads, hist_smem, s>>>(p); break;
+    case 5: fasa_score_kernel<D, 5><<<grid, kScoreThreads, hist_smem, s>>>(p); break;
+    case 6: fasa_score_kernel<D, 6><<<grid, kScoreThreads, hist_smem, s>>>(p); break;
+    case 7: fasa_score_kernel<D, 7><<<grid, kScoreThreads, hist_smem, s>>>(p); break;
+    default: fasa_score_kernel<D, 8><<<grid, kScoreThreads, hist_smem, s>>>(p); break;
+  }
+  fasa_threshold_kernel<<<dim3(p.hq, p.batch), kScanThreads, 0, s>>>(p);
   fasa_scan_kernel<<<dim3(kScanCtas, p.hq, p.batch), kScanThreads, 0, s>>>(p);
   fasa_finish_kernel<<<dim3(p.hq, p.batch), kFinishThreads, 0, s>>>(p);
   fasa_attend_kernel<D><<<dim3(p.n_split, p.hq, p.batch), kAttendWarps * 32, 0, s>>>(p);
@@ -663,6 +701,7 @@ extern "C" atf_status atf_fasa_decode(const void* q_rot, const void* k_chunked, 
   p.cand = reinterpret_cast<uint32_t*>(ws + Lw.cand);
   p.hist = reinterpret_cast<unsigned int*>(ws + Lw.hist);
   p.counts = reinterpret_cast<unsigned int*>(ws + Lw.counts);
+  p.thr = reinterpret_cast<int*>(ws + Lw.thr);
   p.above = reinterpret_cast<int*>(ws + Lw.above);
   p.sel = selected ? selected : reinterpret_cast<int*>(ws + Lw.sel);
   p.partials = reinterpret_cast<float*>(ws + Lw.partials);
