@@ -8,7 +8,7 @@ TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()`` an
 ``bench.py``'s CPU legs, never by the CUDA library.  Plain numpy, one step per
 phase, in the pages' order.
 
-Readings of what the page leaves open (each also listed in the design doc):
+Readings of what the page leaves open:
 - The dominant set is given (calibrating it needs model weights) as a set of
   RoPE frequency pairs; pair i = rotated dims (2i, 2i+1).
 - A token's importance for query head h is the partial dot product of the
