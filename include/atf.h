@@ -269,8 +269,7 @@ atf_status atf_kv_append(const void* k_new, const void* v_new, void* k_cache_chu
  *   scores:    device fp32 [batch][heads][n_cache] or NULL: the scores (entries
  *              n >= kv_len[b] are not written).
  *   workspace: device scratch of atf_fasa_workspace_bytes(...) bytes (the
- *              sizes assume selected and scores are NULL; less is needed when
- *              they are given).
+ *              size assumes selected is NULL; less is needed when it is given).
  * Errors: d not 64/128, more than 8 query heads per kv head, batch above 64,
  * budget outside [1, 4096] -> ATF_ERR_UNSUPPORTED; bad sizes, mask or kv_len,
  * small workspace, null or misaligned pointers -> ATF_ERR_INVALID_ARG. */

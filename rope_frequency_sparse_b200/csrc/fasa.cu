@@ -12,18 +12,22 @@
 //      the kv head.  From +0, every dim of the dominant pairs (ascending) adds
 //      its product with one fp32 fused multiply-add, s <- fl(q_j k_j + s), two
 //      keys at a time as packed f32x2 pairs, so the top-k decision can be
-//      reproduced bit for bit.  The
-//      scores go to memory, with a 4096-bin histogram per query head of the top
-//      12 bits of their order-preserving bit pattern (sign, exponent and three
-//      mantissa bits: a bin spans an eighth of an octave).
+//      reproduced bit for bit.  Each score's order-preserving bit pattern goes
+//      to memory as its top 16 bits (the fp32 score itself only when the caller
+//      asks for it), with a 4096-bin histogram per query head of the top 12
+//      bits (sign, exponent and three mantissa bits: a bin spans an eighth of an
+//      octave).
 //   2. fasa_threshold_kernel (one CTA per row) finds from the histogram the bin
 //      holding the budget-th largest score; fasa_scan_kernel, 32 CTAs per
-//      (query head, sequence), then sweeps 1/32 of the scores each: keys above that bin are in (appended to
-//      an unsorted list), keys in it are candidates.
-//   3. fasa_finish_kernel: one CTA per (query head, sequence).  Radix passes over
-//      the candidates on the rest of the 64-bit selection key (score bits, then
-//      ~index, so equal scores go to the lower index) pick the remaining keys;
-//      the chosen indices are sorted ascending.
+//      (query head, sequence), then sweeps 1/32 of the 16-bit prefixes each:
+//      keys above that bin are in (appended to an unsorted list), keys in it
+//      are candidates.
+//   3. fasa_finish_kernel: one CTA per (query head, sequence).  Recomputes the
+//      candidates' exact scores from the cache in the same order of fused
+//      multiply-adds (the same bits); radix passes over the candidates on the
+//      rest of the 64-bit selection key (score bits, then ~index, so equal
+//      scores go to the lower index) pick the remaining keys; the chosen
+//      indices are sorted ascending.
 //   4. fasa_attend_kernel: (split of 128 selected keys, query head, sequence);
 //      four warps gather the keys' rows from the chunk-major cache and their
 //      values and run an online softmax; partials as in the split decode.
@@ -48,8 +52,7 @@ constexpr int kHistBits = 12;
 constexpr int kHistBins = 1 << kHistBits;
 constexpr int kScanCtas = 32;  // CTAs sweeping one (query head, sequence) row
 constexpr int kScanThreads = 256;
-constexpr int kScanUnroll = 16;
-constexpr int kScanUnroll4 = 4;  // float4 loads in flight per thread
+constexpr int kScanUnroll4 = 4;  // 16-byte loads (8 prefixes each) in flight per thread
 constexpr int kFinishThreads = 1024;
 constexpr int kAttendKeys = 128;  // selected keys per attention split
 constexpr int kAttendWarps = 4;
@@ -62,8 +65,10 @@ struct FasaParams {
   const __nv_bfloat16* kc;  // rotated keys, chunk-major [B][Hkv][d/16][n_cache][16]
   const __nv_bfloat16* v;   // values [B][n_cache][Hkv][d]
   __nv_bfloat16* out;       // [B][Hq][d]
-  float* scores;            // [B][Hq][n_cache]
+  float* scores;            // [B][Hq][n_cache] fp32 scores, or NULL (only written when asked for)
+  uint16_t* pfx;            // [B][Hq][n_pad]: the top 16 bits of each score's order-preserving key
   uint32_t* cand;           // [B][Hq][n_cache] candidates of the threshold bin
+  float* cand_score;        // [B][Hq][n_cache] their exact scores
   unsigned int* hist;       // [B][Hq][kHistBins]
   unsigned int* counts;     // [B][Hq][2]: keys above the threshold bin, candidates
   int* thr;                 // [B][Hq]: the threshold bin
@@ -71,7 +76,7 @@ struct FasaParams {
   int* sel;                 // [B][Hq][budget], ascending, -1 padded
   float* partials;          // [B][Hq][n_split][d + 2]
   int batch, hq, hkv, d, budget, n_split;
-  long long n_cache;
+  long long n_cache, n_pad;  // n_pad: prefix row length, n_cache rounded up to 8
   unsigned long long mask;  // dominant pairs
   long long kv_len[kMaxDecodeBatch];
 };
@@ -161,7 +166,8 @@ __global__ void __launch_bounds__(kScoreThreads, 3) fasa_score_kernel(FasaParams
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       {
-        float* srow = p.scores + (static_cast<long long>(b) * p.hq + kvh * G + g) * p.n_cache;
+        const long long hrow = static_cast<long long>(b) * p.hq + kvh * G + g;
+        uint16_t* prow = p.pfx + hrow * p.n_pad;
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           float sc[2];
@@ -169,8 +175,10 @@ __global__ void __launch_bounds__(kScoreThreads, 3) fasa_score_kernel(FasaParams
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             if (vk[2 * h2 + e]) {
-              srow[nk[2 * h2 + e]] = sc[e];
-              const uint32_t bin = order_key(sc[e]) >> (32 - kHistBits);
+              const uint32_t key = order_key(sc[e]);
+              prow[nk[2 * h2 + e]] = static_cast<uint16_t>(key >> 16);
+              if (p.scores) p.scores[hrow * p.n_cache + nk[2 * h2 + e]] = sc[e];
+              const uint32_t bin = key >> (32 - kHistBits);
               atomicAdd(&shist[g * (kHistBins / 2) + (bin >> 1)], 1u << (16 * (bin & 1u)));
             }
           }
@@ -234,6 +242,29 @@ __device__ __forceinline__ void warp_append(bool flag, uint32_t value, unsigned 
   if (flag && slot < capacity) list[slot] = value;
 }
 
+// The exact score of key n for one query head (q: that head's rotated query as
+// floats), in the scoring kernel's order: dominant dims ascending, one fp32 fused
+// multiply-add each, -0 as +0.
+__device__ __forceinline__ float exact_score(const FasaParams& p, const float* q, const uint4* kbase, long long n) {
+  float s = 0.f;
+  const int nc = p.d / 16;
+  for (int c = 0; c < nc; ++c) {
+    const uint32_t bits = static_cast<uint32_t>((p.mask >> (8 * c)) & 0xFFu);
+    if (!bits) continue;
+    const uint4* row = kbase + (static_cast<long long>(c) * p.n_cache + n) * 2;
+    const uint4 lo = __ldg(row), hi = __ldg(row + 1);
+    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (!((bits >> j) & 1u)) continue;
+      const int dim = 16 * c + 2 * j;
+      s = __fmaf_rn(q[dim], __uint_as_float(w[j] << 16), s);
+      s = __fmaf_rn(q[dim + 1], __uint_as_float(w[j] & 0xFFFF0000u), s);
+    }
+  }
+  return __fadd_rn(s, 0.f);
+}
+
 // The threshold bin of every (query head, sequence) row: the histogram bin holding
 // the need-th largest score (kHistBins when every key is selected: nothing to
 // sweep).  Thread t holds the 16 bins [4096 - 16 (t + 1), 4096 - 16 t), scanned
@@ -282,59 +313,42 @@ __global__ void __launch_bounds__(kScanThreads) fasa_scan_kernel(FasaParams p) {
   const int L = static_cast<int>(p.kv_len[b]);
   const uint32_t thr = static_cast<uint32_t>(p.thr[row]);
   if (thr >= static_cast<uint32_t>(kHistBins)) return;  // every key is selected (or nothing to find)
-  // this CTA's share of the keys (a multiple of 4 long, so that rows of a cache
-  // whose length is a multiple of 4 are read as float4)
-  const int per = ((L + kScanCtas - 1) / kScanCtas + 3) & ~3;
+  // this CTA's share of the keys: a multiple of 8 long, so that 16-byte loads of
+  // 8 prefixes stay aligned (prefix rows are n_pad long, a multiple of 8)
+  const int per = ((L + kScanCtas - 1) / kScanCtas + 7) & ~7;
   const int n_lo = part * per, n_hi = min(L, n_lo + per);
-  const float* sc = p.scores + row * p.n_cache;
+  const uint16_t* prow = p.pfx + row * p.n_pad;
   unsigned int* cnt = p.counts + row * 2;
   uint32_t* above = reinterpret_cast<uint32_t*>(p.above + row * p.budget);
   uint32_t* cand = p.cand + row * p.n_cache;
-  auto visit = [&](int n, float v) {
-    const bool ok = n < n_hi;
-    const uint32_t bin = ok ? order_key(v) >> (32 - kHistBits) : 0u;
-    warp_append(ok && bin > thr, static_cast<uint32_t>(n), &cnt[0], above, static_cast<unsigned int>(p.budget));
-    warp_append(ok && bin == thr, static_cast<uint32_t>(n), &cnt[1], cand, static_cast<unsigned int>(L));
-  };
-  if ((p.n_cache & 3) == 0) {
-    // float4 loads: idx is a multiple of 4 below L <= n_cache, so idx + 3 stays in the row
-    for (int base = n_lo; base < n_hi; base += 4 * kScanThreads * kScanUnroll4) {
-      float4 v[kScanUnroll4];
+  for (int base = n_lo; base < n_hi; base += 8 * kScanThreads * kScanUnroll4) {
+    uint4 v[kScanUnroll4];
 #pragma unroll
-      for (int u = 0; u < kScanUnroll4; ++u) {
-        const int idx = base + 4 * (u * kScanThreads + tid);
-        v[u] = idx < n_hi ? __ldg(reinterpret_cast<const float4*>(sc + idx)) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      // almost every score lies below the threshold bin: one vote per warp skips
-      // the appends unless some lane holds a key at or above it
-      bool hit = false;
+    for (int u = 0; u < kScanUnroll4; ++u) {
+      const int idx = base + 8 * (u * kScanThreads + tid);
+      v[u] = idx < n_hi ? __ldg(reinterpret_cast<const uint4*>(prow + idx)) : make_uint4(0, 0, 0, 0);
+    }
+    // almost every key lies below the threshold bin: each lane marks its keys
+    // above it and in it (bit 8u + e for key 8 * (u * kScanThreads + tid) + e),
+    // and the warp appends only at the positions some lane marked
+    uint32_t am = 0u, cm = 0u;
 #pragma unroll
-      for (int u = 0; u < kScanUnroll4; ++u) {
-        const int idx = base + 4 * (u * kScanThreads + tid);
-        if (idx < n_hi)
-          hit |= max(max(order_key(v[u].x), order_key(v[u].y)), max(order_key(v[u].z), order_key(v[u].w))) >>
-                     (32 - kHistBits) >= thr;
-      }
-      if (!__any_sync(0xffffffffu, hit)) continue;
+    for (int u = 0; u < kScanUnroll4; ++u) {
+      const int idx = base + 8 * (u * kScanThreads + tid);
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
-      for (int u = 0; u < kScanUnroll4; ++u) {
-        const int idx = base + 4 * (u * kScanThreads + tid);
-        visit(idx, v[u].x);
-        visit(idx + 1, v[u].y);
-        visit(idx + 2, v[u].z);
-        visit(idx + 3, v[u].w);
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t bin = (e & 1 ? w[e >> 1] >> 16 : w[e >> 1] & 0xFFFFu) >> 4;
+        const bool ok = idx + e < n_hi;
+        am |= static_cast<uint32_t>(ok && bin > thr) << (8 * u + e);
+        cm |= static_cast<uint32_t>(ok && bin == thr) << (8 * u + e);
       }
     }
-  } else {
-    for (int base = n_lo; base < n_hi; base += kScanThreads * kScanUnroll) {
-      float v[kScanUnroll];
-#pragma unroll
-      for (int u = 0; u < kScanUnroll; ++u) {
-        const int n = base + u * kScanThreads + tid;
-        v[u] = n < n_hi ? __ldg(sc + n) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < kScanUnroll; ++u) visit(base + u * kScanThreads + tid, v[u]);
+    for (uint32_t rest = __reduce_or_sync(0xffffffffu, am | cm); rest; rest &= rest - 1u) {
+      const int j = __ffs(rest) - 1;
+      const uint32_t n = static_cast<uint32_t>(base + 8 * ((j >> 3) * kScanThreads + tid) + (j & 7));
+      warp_append((am >> j) & 1u, n, &cnt[0], above, static_cast<unsigned int>(p.budget));
+      warp_append((cm >> j) & 1u, n, &cnt[1], cand, static_cast<unsigned int>(L));
     }
   }
 }
@@ -342,8 +356,8 @@ __global__ void __launch_bounds__(kScanThreads) fasa_scan_kernel(FasaParams p) {
 __global__ void __launch_bounds__(kFinishThreads) fasa_finish_kernel(FasaParams p) {
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const long long row = static_cast<long long>(b) * p.hq + h;
-  const float* sc = p.scores + row * p.n_cache;
   uint32_t* cand = p.cand + row * p.n_cache;
+  float* cand_score = p.cand_score + row * p.n_cache;
   int* out = p.sel + row * p.budget;
   const int L = static_cast<int>(p.kv_len[b]);
   const int need = L < p.budget ? L : p.budget;
@@ -352,6 +366,7 @@ __global__ void __launch_bounds__(kFinishThreads) fasa_finish_kernel(FasaParams 
   __shared__ unsigned int s_hist[kBins];
   __shared__ int s_warp[kFinishThreads / 32];
   __shared__ int s_nsel, s_total, s_thr, s_above;
+  __shared__ float sq[128];
 
   if (need == L) {  // every key is selected, already in order
     for (int i = tid; i < p.budget; i += kFinishThreads) out[i] = i < L ? i : -1;
@@ -365,16 +380,23 @@ __global__ void __launch_bounds__(kFinishThreads) fasa_finish_kernel(FasaParams 
   if (tid == 0) s_nsel = n_above;
   __syncthreads();
   int left = need - n_above;  // still to choose among the candidates
+  if (left > 0 && left < m) {
+    // the candidates' exact scores, recomputed from the cache in the scoring
+    // kernel's order (the same bits), all candidates in parallel
+    for (int i = tid; i < p.d; i += kFinishThreads) sq[i] = __bfloat162float(p.q[row * p.d + i]);
+    __syncthreads();
+    const uint4* kbase = reinterpret_cast<const uint4*>(p.kc) +
+                         (static_cast<long long>(b) * p.hkv + h / (p.hq / p.hkv)) * (p.d / 16) * p.n_cache * 2;
+    for (int i = tid; i < m; i += kFinishThreads) cand_score[i] = exact_score(p, sq, kbase, cand[i]);
+    __syncthreads();
+  }
   // radix passes over the rest of the selection key: score bits 51..32 below the
   // histogram's 12, then the 32 bits of ~index
   for (int pass = 0; pass < 7 && left > 0 && left < m; ++pass) {
     const int shift = pass < 6 ? 44 - 8 * pass : 0, width = pass < 6 ? 8 : 4;
     for (int i = tid; i < kBins; i += kFinishThreads) s_hist[i] = 0u;
     __syncthreads();
-    for (int i = tid; i < m; i += kFinishThreads) {
-      const uint32_t n = cand[i];
-      atomicAdd(&s_hist[sel_digit(sc[n], n, shift, width)], 1u);
-    }
+    for (int i = tid; i < m; i += kFinishThreads) atomicAdd(&s_hist[sel_digit(cand_score[i], cand[i], shift, width)], 1u);
     __syncthreads();
     if (tid == 0) {
       int above = 0, t = (1 << width) - 1;
@@ -393,9 +415,11 @@ __global__ void __launch_bounds__(kFinishThreads) fasa_finish_kernel(FasaParams 
     for (int base = 0; base < m; base += kFinishThreads) {
       const int i = base + tid;
       uint32_t n = 0, dg = 0;
+      float sv = 0.f;
       if (i < m) {
         n = cand[i];
-        dg = sel_digit(sc[n], n, shift, width);
+        sv = cand_score[i];
+        dg = sel_digit(sv, n, shift, width);
         if (dg > thr) {
           const int slot = atomicAdd(&s_nsel, 1);
           if (slot < need) s_sel[slot] = static_cast<int>(n);
@@ -403,7 +427,10 @@ __global__ void __launch_bounds__(kFinishThreads) fasa_finish_kernel(FasaParams 
       }
       const bool keep = i < m && dg == thr;
       const int rk = block_rank(keep, s_warp, &s_total);  // all reads of this block of cand are done
-      if (keep) cand[kept + rk] = n;
+      if (keep) {
+        cand[kept + rk] = n;
+        cand_score[kept + rk] = sv;
+      }
       kept += s_total;
       __syncthreads();
     }
@@ -575,18 +602,20 @@ __global__ void __launch_bounds__(D) fasa_combine_kernel(FasaParams p) {
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct FasaLayout {
-  size_t scores, cand, hist, counts, thr, above, sel, partials, total;
+  size_t pfx, cand, cand_score, hist, counts, thr, above, sel, partials, total;
 };
 
-FasaLayout fasa_layout(int batch, int heads, long long n_cache, int budget, int d, bool own_scores, bool own_sel) {
+FasaLayout fasa_layout(int batch, int heads, long long n_cache, int budget, int d, bool own_sel) {
   const size_t rows = static_cast<size_t>(batch) * heads;
   const int n_split = (budget + kAttendKeys - 1) / kAttendKeys;
   FasaLayout L{};
   size_t off = 0;
-  L.scores = off;
-  off += own_scores ? 0 : align256(rows * n_cache * sizeof(float));
+  L.pfx = off;
+  off += align256(rows * ((n_cache + 7) / 8 * 8) * sizeof(uint16_t));
   L.cand = off;
   off += align256(rows * n_cache * sizeof(uint32_t));
+  L.cand_score = off;
+  off += align256(rows * n_cache * sizeof(float));
   L.hist = off;  // histograms and counters are cleared together
   off += rows * kHistBins * sizeof(unsigned int);
   L.counts = off;
@@ -656,7 +685,7 @@ using namespace atf;
 
 extern "C" size_t atf_fasa_workspace_bytes(int batch, int heads, long long n_cache, int budget, int d) {
   if (batch <= 0 || heads <= 0 || n_cache <= 0 || budget <= 0 || d <= 0) return 0;
-  return fasa_layout(batch, heads, n_cache, budget, d, false, false).total;
+  return fasa_layout(batch, heads, n_cache, budget, d, false).total;
 }
 
 extern "C" atf_status atf_fasa_decode(const void* q_rot, const void* k_chunked, const void* v, void* out, int batch,
@@ -686,7 +715,7 @@ extern "C" atf_status atf_fasa_decode(const void* q_rot, const void* k_chunked, 
   if (!aligned16(q_rot) || !aligned16(k_chunked) || !aligned16(v) || !aligned16(out) || !aligned16(workspace) ||
       (selected && !aligned16(selected)) || (scores && !aligned16(scores)))
     return report_error(ATF_ERR_INVALID_ARG, "fasa: pointers must be 16-byte aligned");
-  const FasaLayout Lw = fasa_layout(batch, heads, n_cache, budget, d, scores != nullptr, selected != nullptr);
+  const FasaLayout Lw = fasa_layout(batch, heads, n_cache, budget, d, selected != nullptr);
   if (workspace_bytes < Lw.total)
     return report_error(ATF_ERR_INVALID_ARG, "fasa: workspace of %zu bytes needed", Lw.total);
 
@@ -697,7 +726,9 @@ extern "C" atf_status atf_fasa_decode(const void* q_rot, const void* k_chunked, 
   p.kc = static_cast<const __nv_bfloat16*>(k_chunked);
   p.v = static_cast<const __nv_bfloat16*>(v);
   p.out = static_cast<__nv_bfloat16*>(out);
-  p.scores = scores ? scores : reinterpret_cast<float*>(ws + Lw.scores);
+  p.scores = scores;
+  p.pfx = reinterpret_cast<uint16_t*>(ws + Lw.pfx);
+  p.cand_score = reinterpret_cast<float*>(ws + Lw.cand_score);
   p.cand = reinterpret_cast<uint32_t*>(ws + Lw.cand);
   p.hist = reinterpret_cast<unsigned int*>(ws + Lw.hist);
   p.counts = reinterpret_cast<unsigned int*>(ws + Lw.counts);
@@ -712,6 +743,7 @@ extern "C" atf_status atf_fasa_decode(const void* q_rot, const void* k_chunked, 
   p.budget = budget;
   p.n_split = (budget + kAttendKeys - 1) / kAttendKeys;
   p.n_cache = n_cache;
+  p.n_pad = (n_cache + 7) / 8 * 8;
   p.mask = pair_mask;
   for (int b = 0; b < batch; ++b) p.kv_len[b] = kv_len[b];
   cudaError_t e = cudaMemsetAsync(p.hist, 0, Lw.above - Lw.hist, s);  // histograms and counters

@@ -168,12 +168,12 @@ def test_workspace_sizes(lib):
     assert hws == 3 * qb + 3 * kb
     assert atf.atf_prefill_host_workspace_bytes(2, 1000, 1500, 28, 4, 128, 1) == 2 * qb + 2 * kb
     assert atf.atf_prefill_host_workspace_bytes(0, 1000, 1500, 28, 4, 128, 0) == 0
-    # FASA: scores + candidates per (sequence, query head, key), 4096-bin histograms,
+    # FASA: 16-bit score prefixes, candidates and their scores per (sequence, query head, key), 4096-bin histograms,
     # two counters and the threshold bin (each padded to 256 bytes), the above-threshold and the selected
     # indices, attention partials (128 selected keys per split)
     fws = atf.atf_fasa_workspace_bytes(4, 28, 1 << 20, 2048, 128)
     rows = 4 * 28
-    assert fws == rows * (1 << 20) * 8 + rows * 4096 * 4 + 1024 + 512 + 2 * rows * 2048 * 4 + rows * 16 * 130 * 4
+    assert fws == rows * (1 << 20) * 10 + rows * 4096 * 4 + 1024 + 512 + 2 * rows * 2048 * 4 + rows * 16 * 130 * 4
     dws = atf.atf_decode_workspace_bytes(4, 28, 4, 1 << 20, 128)
     assert dws % (4 * 28 * 130 * 4) == 0 and dws > 0
 
