@@ -134,6 +134,27 @@ struct WarpWindows {
   }
 };
 
+// The 32 key words of one pair (columns c_lo .. c_lo+31) in a 128-byte-swizzled
+// K tile: column cc at kb[cc % 8] + 128 cc.
+template <int CC>
+__device__ __forceinline__ void load_key_words(uint32_t (&kw)[32], const uint32_t (&kb)[8]) {
+  if constexpr (CC < 32) {
+    kw[CC] = lds32_at<CC * 128>(kb[CC & 7]);
+    load_key_words<CC + 1>(kw, kb);
+  }
+}
+
+// Adds (q_2i k_2i + q_2i+1 k_2i+1)(cc), q signed, to the columns cc of the chunk
+// whose bit of `mask` is set.
+template <int CC>
+__device__ __forceinline__ void correct_columns(float (&x)[32], const uint32_t (&kw)[32], uint32_t mask,
+                                                uint32_t qs) {
+  if constexpr (CC < 32) {
+    x[CC] = fma_bf16x2_f32_if<CC>(mask, qs, kw[CC], x[CC]);
+    correct_columns<CC + 1>(x, kw, mask, qs);
+  }
+}
+
 // Byte offset of pair i (4 bytes) of row r inside a 128-row tile stored as
 // 64-dim boxes with the 128-byte swizzle (16-byte chunk index XOR row % 8).
 __device__ __forceinline__ uint32_t pair_offset(int r, int i) {
@@ -512,55 +533,57 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                   for (int cc = 0; cc < 32; ++cc) x[cc] = 0.f;
                 }
-                // Each pair of the chunk in turn.  Its key words (k_2i(c), k_2i+1(c))
-                // for the chunk's 32 columns are read straight from the K tile: the
-                // address depends only on the column, so every lane issues the same
-                // 32 broadcast loads, with no staging and no warp synchronisation.
-#pragma unroll 1
-                while (tbits) {
-                  const int k = __ffs(tbits) - 1;
-                  tbits &= tbits - 1;
-                  const int i = hb + k;
-                  uint32_t qp = 0u;
+                // The key words (k_2i(c), k_2i+1(c)) of the chunk's 32 columns are read
+                // straight from the K tile: the address depends only on the column, so
+                // every lane issues the same broadcast loads, with no staging and no
+                // warp synchronisation.
+                // this row's (q_2i, q_2i+1) as a bf16x2 word: from Q~ while the pair is
+                // issued, else from the stash of recently zeroed pairs, else from memory
+                auto load_qpair = [&](int i) -> uint32_t {
+                  uint32_t qv = 0u;
                   if (row_ok) {
                     if (i >= z)
-                      qp = lds32(q_base + pair_offset(r, i));
+                      qv = lds32(q_base + pair_offset(r, i));
                     else if (static_cast<unsigned>(i - zst) < static_cast<unsigned>(kStash))
-                      qp = lds32(stash_base + static_cast<uint32_t>((i - zst) * BM) * 4u);
+                      qv = lds32(stash_base + static_cast<uint32_t>((i - zst) * BM) * 4u);
                     else
-                      qp = __ldg(qrow + i);
+                      qv = __ldg(qrow + i);
                   }
+                  return qv;
+                };
+                int k = __ffs(tbits) - 1;
+                tbits &= tbits - 1;
+                uint32_t qp = load_qpair(hb + k);
+#pragma unroll 1
+                while (true) {
+                  const int i = hb + k;
+                  // column cc's key word sits at kb[cc % 8] + 128 cc (the swizzle
+                  // permutes the 16-byte chunks of a row by row % 8)
                   const uint32_t kp = kbase + (i >> 5) * (BN * 128) + c_lo * 128 + (i & 3) * 4;
                   const uint32_t ci = static_cast<uint32_t>((i & 31) >> 2);
+                  uint32_t kb[8];
+#pragma unroll
+                  for (int sw = 0; sw < 8; ++sw) kb[sw] = kp + ((ci ^ sw) << 4);
                   uint32_t kw[32];
-#pragma unroll
-                  for (int cc = 0; cc < 32; ++cc) kw[cc] = lds32(kp + cc * 128 + ((ci ^ (cc & 7)) << 4));
+                  load_key_words<0>(kw, kb);
                   const int wi = __shfl_sync(0xffffffffu, wl, k);
-                  const bool add = i < z;  // zeroed pair: add back where c >= tl; else subtract where c < tl
-                  const float sg = add ? 1.f : -1.f;
-                  const uint64_t qa2 = pack2(sg * bf16lo_to_f32(qp), sg * bf16lo_to_f32(qp));
-                  const uint64_t qb2 = pack2(sg * bf16hi_to_f32(qp), sg * bf16hi_to_f32(qp));
-                  if ((fbits >> k) & 1u) {  // every row of the warp corrects the whole chunk
-#pragma unroll
-                    for (int cp = 0; cp < 16; ++cp) {
-                      uint64_t x2 = pack2(x[2 * cp], x[2 * cp + 1]);
-                      x2 = ffma2(qa2, pack2(bf16lo_to_f32(kw[2 * cp]), bf16lo_to_f32(kw[2 * cp + 1])), x2);
-                      x2 = ffma2(qb2, pack2(bf16hi_to_f32(kw[2 * cp]), bf16hi_to_f32(kw[2 * cp + 1])), x2);
-                      unpack2(x2, x[2 * cp], x[2 * cp + 1]);
-                    }
-                  } else {
-                    const int tc = r + cen - wi - c_lo;  // chunk columns cc < tc lie outside the window
-#pragma unroll
-                    for (int cp = 0; cp < 16; ++cp) {
-                      uint64_t y2 = pack2(x[2 * cp], x[2 * cp + 1]);
-                      y2 = ffma2(qa2, pack2(bf16lo_to_f32(kw[2 * cp]), bf16lo_to_f32(kw[2 * cp + 1])), y2);
-                      y2 = ffma2(qb2, pack2(bf16hi_to_f32(kw[2 * cp]), bf16hi_to_f32(kw[2 * cp + 1])), y2);
-                      float y0, y1;
-                      unpack2(y2, y0, y1);
-                      if ((2 * cp >= tc) == add) x[2 * cp] = y0;
-                      if ((2 * cp + 1 >= tc) == add) x[2 * cp + 1] = y1;
-                    }
+                  const bool more = tbits != 0u;
+                  int kn = 0;
+                  uint32_t qpn = 0u;
+                  if (more) {  // the next item's query pair, in flight during this one
+                    kn = __ffs(tbits) - 1;
+                    tbits &= tbits - 1;
+                    qpn = load_qpair(hb + kn);
                   }
+                  const bool add = i < z;  // zeroed pair: add back where cc >= tc; else subtract where cc < tc
+                  const uint32_t qs = add ? qp : (qp ^ 0x80008000u);  // both bf16 halves negated to subtract
+                  const int tc = r + cen - wi - c_lo;  // chunk columns cc < tc lie outside the window
+                  const uint32_t ge = tc <= 0 ? ~0u : (tc >= 32 ? 0u : (~0u << tc));
+                  const uint32_t mk = ((fbits >> k) & 1u) ? ~0u : (add ? ge : ~ge);
+                  correct_columns<0>(x, kw, mk, qs);
+                  if (!more) break;
+                  k = kn;
+                  qp = qpn;
                 }
                 tmem_st32(s_tmem + c_lo, reinterpret_cast<uint32_t*>(x));
                 s_chunks |= 1u << qc;

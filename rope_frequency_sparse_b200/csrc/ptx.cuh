@@ -308,5 +308,26 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
+// Shared-memory load at a compile-time byte offset from `addr`.
+template <int OFF>
+__device__ __forceinline__ uint32_t lds32_at(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(OFF));
+  return v;
+}
+// x + q_lo k_lo + q_hi k_hi for two bf16x2 words, in that order (each step one fp32
+// fused multiply-add of the exactly widened bf16 operands) where bit BIT of
+// `mask` is set; x unchanged where it is clear.
+template <int BIT>
+__device__ __forceinline__ float fma_bf16x2_f32_if(uint32_t mask, uint32_t q, uint32_t k, float x) {
+  float d = x;
+  asm("{\n\t.reg .b16 ql, qh, kl, kh;\n\t.reg .pred pp;\n\t.reg .b32 t;\n\t"
+      "and.b32 t, %1, %4;\n\tsetp.ne.u32 pp, t, 0;\n\t"
+      "mov.b32 {ql, qh}, %2;\n\tmov.b32 {kl, kh}, %3;\n\t"
+      "@pp fma.rn.f32.bf16 %0, ql, kl, %0;\n\t@pp fma.rn.f32.bf16 %0, qh, kh, %0;\n\t}"
+      : "+f"(d)
+      : "r"(mask), "r"(q), "r"(k), "n"(1u << BIT));
+  return d;
+}
 
 }  // namespace atf
