@@ -54,7 +54,8 @@ namespace {
 
 constexpr int BM = 128;        // query rows per Q tile (MMA M, TMEM lanes)
 constexpr int NQ = 2;          // Q tiles per CTA
-constexpr int BN = 128;        // keys per KV tile
+constexpr int BN = 128;        // keys per KV tile (four 32-column chunks)
+static_assert(BN == 128, "the correction code selects among four 32-column chunks");
 constexpr int kThreads = 384;  // 12 warps = 3 warpgroups
 constexpr int kRegsLaunch = 168;   // registers per thread at launch (checked by the launcher)
 constexpr int kRegsCtl = 64;       // warpgroup 0 after reallocation
@@ -486,44 +487,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nv = cmax + 1;  // valid columns of this row
         if (SPARSE) cnt += static_cast<unsigned long long>(a) * nv;
         const int cmax_w = (SPARSE && a < u) ? __reduce_max_sync(0xffffffffu, cmax) : 0;
+        // Classification of pairs hb .. hb+31 (lane l: pair hb + l) for this warp's
+        // rows: per 32-column chunk, the pairs some row must correct (tb) and those
+        // every row corrects entirely (fb).  Chunks past every row's last valid column
+        // (beyond the causal diagonal or the last key, cmax_w) are masked out whole:
+        // nothing there needs correcting.  For pairs in [a, u) the windows lie within
+        // 127 of the centre, so the thresholds fit in 32 bits.
+        const int cw = SPARSE ? quarter * 32 + static_cast<int>(center) : 0;  // threshold offset of row 0 of the warp
+        auto classify = [&](int hb, int& wl, uint32_t (&tb)[BN / 32], uint32_t (&fb)[BN / 32]) {
+          const int il = hb + lane;
+          const bool valid = il < u;
+          wl = valid ? sh->w[il] : 0;
+          const int twl = cw - wl;  // smallest threshold among the warp's rows
+          const bool addl = il < z;
+#pragma unroll
+          for (int qc = 0; qc < BN / 32; ++qc) {
+            const int c_lo = 32 * qc;
+            tb[qc] = __ballot_sync(0xffffffffu,
+                                   valid && c_lo <= cmax_w && (addl ? (c_lo + 31 >= twl) : (c_lo < twl + 31)));
+            fb[qc] = __ballot_sync(0xffffffffu, valid && (addl ? (c_lo >= twl + 31) : (c_lo + 31 < twl)));
+          }
+        };
+        // the first batch is classified before S arrives, off the softmax -> MMA chain
+        int wl0 = 0;
+        uint32_t tb0[BN / 32] = {}, fb0[BN / 32] = {};
+        if (SPARSE && a < u) classify(a, wl0, tb0, fb0);
         if (!(ok = warp_wait(&sh->s_full[g], (j - j0) & 1, abort, p.err, 0x303))) break;
         tc_fence_after();
         uint32_t s_chunks = has_mma ? 0xFu : 0u;  // 32-column chunks of S held in TMEM
         if (SPARSE) {
           if (__builtin_expect(a < u, 0)) {
             // ---- boundary corrections, in place on S in TMEM, 32 columns at a time.
-            // For pairs in [a, u) the windows lie within 127 of the centre, so the
-            // thresholds fit in 32 bits.
             const int cen = static_cast<int>(center);
-            const int cw = quarter * 32 + cen;  // threshold offset of the warp's first row
             const uint32_t kbase = smem_u32(sK + s * C::TILE_BYTES);
             const uint32_t q_base = smem_u32(sQg);
             const uint32_t stash_base = smem_u32(&sh->stash[g][0][r]);
-            // chunks past every row's last valid column (beyond the causal diagonal
-            // or the last key, cmax_w) are masked out whole: nothing there needs correcting
 #pragma unroll 1
             for (int hb = a; hb < u; hb += 32) {
-              // classify pair hb + lane: the chunks some row of this warp must
-              // correct (tm), and those every row corrects entirely (fm)
-              const int il = hb + lane;
-              const bool valid = il < u;
-              const int wl = valid ? sh->w[il] : 0;
-              const int twl = cw - wl;  // smallest threshold among the warp's rows
-              const bool addl = il < z;
-              uint32_t tm = 0u, fm = 0u;
+              int wl = wl0;
+              uint32_t tb[BN / 32], fb[BN / 32];
 #pragma unroll
               for (int qc = 0; qc < BN / 32; ++qc) {
-                const int c_lo = 32 * qc;
-                const bool touch = valid && c_lo <= cmax_w && (addl ? (c_lo + 31 >= twl) : (c_lo < twl + 31));
-                const bool fullc = valid && (addl ? (c_lo >= twl + 31) : (c_lo + 31 < twl));
-                tm |= static_cast<uint32_t>(touch) << qc;
-                fm |= static_cast<uint32_t>(fullc) << qc;
+                tb[qc] = tb0[qc];
+                fb[qc] = fb0[qc];
               }
+              if (hb != a) classify(hb, wl, tb, fb);
 #pragma unroll 1
               for (int qc = 0; qc < BN / 32; ++qc) {
                 const int c_lo = 32 * qc;
-                uint32_t tbits = __ballot_sync(0xffffffffu, (tm >> qc) & 1u);
-                const uint32_t fbits = __ballot_sync(0xffffffffu, (fm >> qc) & 1u);
+                uint32_t tbits = qc == 0 ? tb[0] : qc == 1 ? tb[1] : qc == 2 ? tb[2] : tb[3];
+                const uint32_t fbits = qc == 0 ? fb[0] : qc == 1 ? fb[1] : qc == 2 ? fb[2] : fb[3];
                 if (!tbits) continue;
                 float x[32];
                 if ((s_chunks >> qc) & 1u) {
