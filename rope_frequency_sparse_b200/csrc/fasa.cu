@@ -53,6 +53,7 @@ constexpr int kHistBins = 1 << kHistBits;
 constexpr int kScanCtas = 32;  // CTAs sweeping one (query head, sequence) row
 constexpr int kScanThreads = 256;
 constexpr int kScanUnroll4 = 4;  // 16-byte loads (8 prefixes each) in flight per thread
+constexpr int kScanStage = 1024;  // per scan CTA, list entries staged in shared memory before the global append
 constexpr int kFinishThreads = 1024;
 constexpr int kAttendKeys = 128;  // selected keys per attention split
 constexpr int kAttendWarps = 4;
@@ -227,19 +228,26 @@ __device__ __forceinline__ uint32_t sel_digit(float score, uint32_t n, int shift
   return static_cast<uint32_t>(key >> shift) & ((1u << width) - 1u);
 }
 
-// Appends the lanes' values where `flag` holds to list[] at slots taken from
-// *counter, one atomic per warp; slots at or past `capacity` are counted but not
-// written.
-__device__ __forceinline__ void warp_append(bool flag, uint32_t value, unsigned int* counter, uint32_t* list,
-                                            unsigned int capacity) {
+// Appends the lanes' values where `flag` holds to a shared-memory list of
+// kScanStage entries, slots taken from *s_count with one atomic per warp; a lane
+// whose slot lies past the list appends to the global list itself (slots at or past
+// `capacity` are counted but not written).
+__device__ __forceinline__ void warp_append_staged(bool flag, uint32_t value, unsigned int* s_count, uint32_t* s_list,
+                                                   unsigned int* counter, uint32_t* list, unsigned int capacity) {
   const int lane = threadIdx.x & 31;
   const uint32_t bal = __ballot_sync(0xffffffffu, flag);
   if (!bal) return;
   unsigned int base = 0;
-  if (lane == __ffs(bal) - 1) base = atomicAdd(counter, static_cast<unsigned int>(__popc(bal)));
+  if (lane == __ffs(bal) - 1) base = atomicAdd(s_count, static_cast<unsigned int>(__popc(bal)));
   base = __shfl_sync(0xffffffffu, base, __ffs(bal) - 1);
   const unsigned int slot = base + __popc(bal & ((1u << lane) - 1u));
-  if (flag && slot < capacity) list[slot] = value;
+  if (!flag) return;
+  if (slot < static_cast<unsigned int>(kScanStage)) {
+    s_list[slot] = value;
+  } else {
+    const unsigned int g = atomicAdd(counter, 1u);
+    if (g < capacity) list[g] = value;
+  }
 }
 
 // The exact score of key n for one query head (q: that head's rotated query as
@@ -321,6 +329,12 @@ __global__ void __launch_bounds__(kScanThreads) fasa_scan_kernel(FasaParams p) {
   unsigned int* cnt = p.counts + row * 2;
   uint32_t* above = reinterpret_cast<uint32_t*>(p.above + row * p.budget);
   uint32_t* cand = p.cand + row * p.n_cache;
+  // the CTA's entries of both lists gather in shared memory; one global atomic per
+  // list reserves their slots at the end
+  __shared__ uint32_t s_above[kScanStage], s_cand[kScanStage];
+  __shared__ unsigned int s_na, s_nc, s_ga, s_gc;
+  if (tid == 0) s_na = s_nc = 0u;
+  __syncthreads();
   for (int base = n_lo; base < n_hi; base += 8 * kScanThreads * kScanUnroll4) {
     uint4 v[kScanUnroll4];
 #pragma unroll
@@ -347,10 +361,22 @@ __global__ void __launch_bounds__(kScanThreads) fasa_scan_kernel(FasaParams p) {
     for (uint32_t rest = __reduce_or_sync(0xffffffffu, am | cm); rest; rest &= rest - 1u) {
       const int j = __ffs(rest) - 1;
       const uint32_t n = static_cast<uint32_t>(base + 8 * ((j >> 3) * kScanThreads + tid) + (j & 7));
-      warp_append((am >> j) & 1u, n, &cnt[0], above, static_cast<unsigned int>(p.budget));
-      warp_append((cm >> j) & 1u, n, &cnt[1], cand, static_cast<unsigned int>(L));
+      warp_append_staged((am >> j) & 1u, n, &s_na, s_above, &cnt[0], above, static_cast<unsigned int>(p.budget));
+      warp_append_staged((cm >> j) & 1u, n, &s_nc, s_cand, &cnt[1], cand, static_cast<unsigned int>(L));
     }
   }
+  __syncthreads();
+  const unsigned int na = min(s_na, static_cast<unsigned int>(kScanStage));
+  const unsigned int nc = min(s_nc, static_cast<unsigned int>(kScanStage));
+  if (tid == 0) {
+    s_ga = na ? atomicAdd(&cnt[0], na) : 0u;
+    s_gc = nc ? atomicAdd(&cnt[1], nc) : 0u;
+  }
+  __syncthreads();
+  for (unsigned int i = tid; i < na; i += kScanThreads)
+    if (s_ga + i < static_cast<unsigned int>(p.budget)) above[s_ga + i] = s_above[i];
+  for (unsigned int i = tid; i < nc; i += kScanThreads)
+    if (s_gc + i < static_cast<unsigned int>(L)) cand[s_gc + i] = s_cand[i];
 }
 
 __global__ void __launch_bounds__(kFinishThreads) fasa_finish_kernel(FasaParams p) {

@@ -73,6 +73,25 @@ def test_fasa_heavy_ties_use_every_radix_pass():
     assert (sel >= 0).all()
 
 
+def test_fasa_lists_longer_than_a_scan_block_stages():
+    """65536 keys, 2048 per scan block: head 0 scores every key alike (all are
+    candidates), head 1 scores keys 0..2999 high (they are all above the threshold
+    bin, 2048 of them in one block), so both lists overflow a block's shared-memory
+    stage and spill to the global append."""
+    B, N, Hq, Hkv, d = 1, 1 << 16, 2, 1, 64
+    g = np.random.default_rng(9)
+    q = torch.zeros(B, Hq, d)
+    q[:, :, 2 * 7] = 1.0
+    k = torch.zeros(B, N, Hkv, d)
+    k[0, :, 0, 2 * 7] = 1.0
+    k[0, :3000, 0, 2 * 7 + 1] = 2.0
+    q[:, 1, 2 * 7 + 1] = 1.0
+    v = torch.from_numpy(g.standard_normal((B, N, Hkv, d)).astype(np.float32))
+    q, k, v = q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+    sel = _check(q, k, v, [N], 1 << 7, 4000)
+    assert (sel[0, 0] == np.arange(4000)).all() and (sel[0, 1] == np.arange(4000)).all()
+
+
 def test_fasa_without_optional_outputs_gives_the_same_result():
     q, k, v = _inputs(2, 4096, 8, 2, 128, seed=67)
     kv_len, budget = [4096, 2500], 300
