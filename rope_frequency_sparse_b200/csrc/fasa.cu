@@ -424,15 +424,35 @@ __global__ void __launch_bounds__(kFinishThreads) fasa_finish_kernel(FasaParams 
     __syncthreads();
     for (int i = tid; i < m; i += kFinishThreads) atomicAdd(&s_hist[sel_digit(cand_score[i], cand[i], shift, width)], 1u);
     __syncthreads();
-    if (tid == 0) {
-      int above = 0, t = (1 << width) - 1;
-      for (; t > 0; --t) {
-        const int c = static_cast<int>(s_hist[t]);
-        if (above + c >= left) break;
-        above += c;
+    if (tid < 32) {
+      // the threshold digit: the largest t with #(digits >= t) >= left (t = 0 at the
+      // latest, since m > left), and the count above it; one warp, each lane a run
+      // of consecutive digits, suffix sums across the lanes
+      const int nb = 1 << width, per = (nb + 31) / 32, lo = tid * per;
+      int lsum = 0;
+      for (int u = lo; u < lo + per && u < nb; ++u) lsum += static_cast<int>(s_hist[u]);
+      int suf = lsum;  // digits >= lo
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_down_sync(0xffffffffu, suf, off);
+        if (tid + off < 32) suf += y;
       }
-      s_thr = t;
-      s_above = above;
+      int t = -1, above = 0;
+      int run = suf - lsum;  // digits past this lane's run
+      for (int u = min(lo + per, nb) - 1; u >= lo; --u) {
+        const int c = static_cast<int>(s_hist[u]);
+        if (run + c >= left) {
+          t = u;
+          above = run;
+          break;
+        }
+        run += c;
+      }
+      const int tmax = __reduce_max_sync(0xffffffffu, t);
+      if (t == tmax && t >= 0) {  // one lane holds it
+        s_thr = t;
+        s_above = above;
+      }
     }
     __syncthreads();
     const uint32_t thr = static_cast<uint32_t>(s_thr);
