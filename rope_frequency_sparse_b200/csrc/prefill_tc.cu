@@ -29,14 +29,16 @@
 // Window structure.  W is non-decreasing in i (wavelengths grow), so the active
 // pairs of any element form a suffix {i >= i*(Delta)}.  KV tiles are visited
 // from the diagonal towards key 0, so a Q tile's centre distance c = m0 - n0
-// grows monotonically.  Pairs with W_i < c are zeroed in that Q tile's shared-
-// memory copy once and for all, and whole 8-pair chunks below the first
-// non-zeroed pair are not issued to the MMA (the contraction depth shrinks tile
-// by tile).  Elements of a tile that straddles a window boundary are fixed on the
-// CUDA cores before the softmax reads S: a zeroed pair whose window still covers
-// the element is added back, an issued pair whose window does not is subtracted;
-// only straddling pairs, and only 32-column chunks a warp's rows reach, are
-// touched.  The per-tile pair ranges are tabulated in shared memory at the start.
+// grows monotonically.  Each warp (32 rows) zeroes, in its rows of the Q tile's
+// shared-memory copy, the pairs whose windows end before about the median
+// distance its rows see on the tile, once and for all, and whole 8-pair chunks
+// zeroed in every row are not issued to the MMA (the contraction depth shrinks
+// tile by tile).  Elements of a tile that straddles a window boundary are fixed on
+// the CUDA cores before the softmax reads S: a zeroed pair whose window still
+// covers the element is added back, an issued pair whose window does not is
+// subtracted; only straddling pairs, and only 32-column chunks a warp's rows
+// reach, are touched.  The window counts come from the W table held across each
+// warp's lanes (ballots), with no per-tile table.
 //
 // Exponentials.  The SFU evaluates 16 ex2 per clock per SM, as many as the
 // tensor core needs cycles for a 128x128 tile's two MMAs.  A share of the column
