@@ -30,6 +30,9 @@
  *     for decode; theta > 1; alpha > 0 (finite or +inf).
  *   - Errors: a non-zero atf_status; atf_last_error() gives the message of the
  *     last failing call on the calling thread.
+ *   - The library looks up the device address of its error word once per device
+ *     and keeps it for the process: do not call it again on a device after a
+ *     cudaDeviceReset of that device.
  */
 #ifndef ATF_H
 #define ATF_H
@@ -180,7 +183,9 @@ size_t atf_decode_workspace_bytes(int batch, int heads, int kv_heads, long long 
  *   workspace, skipped_pairs: as in atf_decode (workspace sized with
  *   atf_decode_workspace_bytes for the largest n_keys).
  *   n_keys, key_pos0, q_pos: HOST arrays of batch entries; n_keys[b] may be 0 (an
- *   empty piece merges as nothing).
+ *   empty piece merges as nothing).  q_pos[b] - key_pos0[b] must be below 2^31
+ *   (the kernels hold distances and windows in 32 bits); a larger distance is
+ *   rejected with ATF_ERR_UNSUPPORTED before any work.
  *   partial: DEVICE fp32 [batch][heads][d + 2]: the piece's softmax numerator
  *   (relative to its maximum), its maximum logit (log2 units, -inf when empty)
  *   and its row sum: the form atf_decode_merge reads. */
@@ -212,7 +217,10 @@ atf_status atf_decode_merge(const float* partials, int n_parts, int batch, int h
  *     exits.  The first call on a device looks up its device address
  *     (cudaGetSymbolAddress, with that device current) and caches it; make that
  *     first call before any stream capture.  It calls no cudaMalloc, cudaFree or
- *     other allocating routine.
+ *     other allocating routine.  The cached address belongs to the device's
+ *     current context: it does not survive cudaDeviceReset (or any other
+ *     destruction of that context), after which this entry point must not be
+ *     called again in the same process.
  *   - All calls on a device share the array and it keeps the previous call's
  *     contents (every value read is written first in the same call).  Calls whose
  *     kernels overlap on the GPU (e.g. on unordered streams) race on it. */

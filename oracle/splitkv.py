@@ -34,10 +34,11 @@ def _f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
-def partial(q, k_rot, v, lo, hi, q_pos, theta: float, alpha: float) -> np.ndarray:
+def partial(q, k_rot, v, lo, hi, q_pos, theta: float, alpha: float, key_pos0=None) -> np.ndarray:
     """Partials [B][Hq][d + 2] of raw queries q [B][Hq][d] (rotated here at
-    q_pos[b]) against keys lo[b] .. hi[b]-1 of k_rot / v [B][N][Hkv][d] (key n
-    rotated at position n)."""
+    q_pos[b]) against keys lo[b] .. hi[b]-1 of k_rot / v [B][N][Hkv][d]: key n
+    sits at position key_pos0[b] + n (key_pos0 None: position n) and was rotated
+    there."""
     qq = _f64(q)
     k = _f64(k_rot)
     vv = _f64(v)
@@ -52,7 +53,8 @@ def partial(q, k_rot, v, lo, hi, q_pos, theta: float, alpha: float) -> np.ndarra
         if n.size == 0:
             out[b, :, d] = -np.inf
             continue
-        delta = int(q_pos[b]) - n
+        p0 = 0 if key_pos0 is None else int(key_pos0[b])
+        delta = int(q_pos[b]) - (p0 + n)
         active = W[None, :] >= delta[:, None]  # [keys][pairs]
         for h in range(Hq):
             kk = k[b, n, h // G, :]

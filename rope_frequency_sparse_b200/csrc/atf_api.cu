@@ -378,6 +378,11 @@ atf_status decode_impl(const void* q, const void* k_chunked, const void* v, void
     if (p0 < 0 || qp < 0 || qp < p0 + n_keys[b] - 1 || qp > (1LL << 40))
       return fail(ATF_ERR_INVALID_ARG, "decode: sequence %d: the query (position %lld) must not precede its keys "
                   "(positions %lld ..%lld)", b, qp, p0, p0 + n_keys[b] - 1);
+    // the kernels hold windows and distances in 32 bits (W_i clamped to 2^31-1):
+    // every query-key distance must stay below 2^31 for that clamp to be exact
+    if (qp - p0 > 0x7fffffffLL)
+      return fail(ATF_ERR_UNSUPPORTED, "decode: sequence %d: the query (position %lld) is 2^31 or more positions "
+                  "after its first key (position %lld)", b, qp, p0);
     if (n_keys[b] > max_len) max_len = n_keys[b];
   }
   const size_t need = atf_decode_workspace_bytes(batch, heads, kv_heads, max_len, d);

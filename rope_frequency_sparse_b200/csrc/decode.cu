@@ -31,6 +31,8 @@
 // second kernel merges the partials.
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 #include "atf_internal.cuh"
 #include "ptx.cuh"
 
@@ -450,11 +452,13 @@ static cudaError_t launch_dec(const DecodeParams& p, const CUtensorMap& tv, cons
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  static unsigned long long configured = 0;  // one bit per device
-  if (dev < 64 && !(configured & (1ull << dev))) {
+  // one bit per device; setting the attribute twice (two threads racing on the
+  // first call) is harmless, the atomic keeps the bit updates themselves defined
+  static std::atomic<unsigned long long> configured{0};
+  if (dev >= 64 || !(configured.load(std::memory_order_acquire) & (1ull << dev))) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    configured |= 1ull << dev;
+    if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_acq_rel);
   }
   kern<<<dim3(p.n_split, p.hkv, p.batch), kDecThreads, bytes, s>>>(tv, tk, p);
   return cudaGetLastError();

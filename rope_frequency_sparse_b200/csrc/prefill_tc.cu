@@ -47,6 +47,8 @@
 // compile-time mask, off by default (see ATF_EXP_FMA_MASK).
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 #include "atf_internal.cuh"
 #include "ptx.cuh"
 
@@ -774,8 +776,10 @@ static cudaError_t launch_tc(const PrefillParams& p, const CUtensorMap& tq, cons
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  static unsigned long long configured = 0;  // one bit per device
-  if (dev < 64 && !(configured & (1ull << dev))) {
+  // one bit per device; two threads racing on the first call both check and set
+  // the attribute, which is harmless, and the atomic keeps the bit updates defined
+  static std::atomic<unsigned long long> configured{0};
+  if (dev >= 64 || !(configured.load(std::memory_order_acquire) & (1ull << dev))) {
     // The register reallocation inside the kernel needs exactly the launch
     // allocation it was written for; anything else could leave setmaxnreg.inc
     // waiting, so refuse to launch.
@@ -785,7 +789,7 @@ static cudaError_t launch_tc(const PrefillParams& p, const CUtensorMap& tq, cons
     if (attr.numRegs != kRegsLaunch) return cudaErrorInvalidKernelImage;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    configured |= 1ull << dev;
+    if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_acq_rel);
   }
   const long long nqt = (p.q_len + BM - 1) / BM;
   const long long ctas = (nqt + NQ - 1) / NQ * p.hq * p.batch;

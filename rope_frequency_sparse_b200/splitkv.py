@@ -12,6 +12,7 @@ a far one, so the ranges near the query are shorter.
 """
 from __future__ import annotations
 
+import contextlib
 import math
 
 import numpy as np
@@ -60,6 +61,18 @@ def _gpu_partial(q, kc, v, n_keys, key_pos0, q_pos, theta, alpha, pairing, strea
     return part
 
 
+def _torch_stream(stream, device):
+    """The torch stream object for a stream argument of the binding (None: torch's
+    current stream, an int: a raw cudaStream_t handle, else a torch stream)."""
+    import torch
+
+    if stream is None:
+        return None
+    if isinstance(stream, int):
+        return torch.cuda.ExternalStream(stream, device=device)
+    return stream
+
+
 def _gpu_merge(parts, world, B, Hq, d, stream):
     import torch
 
@@ -87,13 +100,18 @@ def decode_split_kv(q, kc_local, v_local, n_keys_local, key_pos0, q_pos, theta, 
     part = (partial_fn or _gpu_partial)(q, kc_local, v_local, list(n_keys_local), list(key_pos0), list(q_pos),
                                        theta, alpha, pairing, stream)
     if world > 1:
-        if dist.get_backend(group) == "nccl":
-            gathered = torch.empty((world,) + tuple(part.shape), dtype=part.dtype, device=part.device)
-            dist.all_gather_into_tensor(gathered, part.contiguous(), group=group)
-        else:
-            pieces = [torch.empty_like(part) for _ in range(world)]
-            dist.all_gather(pieces, part.contiguous(), group=group)
-            gathered = torch.stack(pieces)
+        # the partial was written on `stream`: issue the exchange on that stream too,
+        # so the gather reads the partial only after the kernel that writes it, and
+        # the merge (also on `stream`) reads the gathered parts only after the gather
+        ts = _torch_stream(stream, part.device) if part.is_cuda else None
+        with (torch.cuda.stream(ts) if ts is not None else contextlib.nullcontext()):
+            if dist.get_backend(group) == "nccl":
+                gathered = torch.empty((world,) + tuple(part.shape), dtype=part.dtype, device=part.device)
+                dist.all_gather_into_tensor(gathered, part.contiguous(), group=group)
+            else:
+                pieces = [torch.empty_like(part) for _ in range(world)]
+                dist.all_gather(pieces, part.contiguous(), group=group)
+                gathered = torch.stack(pieces)
     else:
         gathered = part[None]
     return (merge_fn or _gpu_merge)(gathered, world, B, Hq, d, stream)

@@ -99,6 +99,11 @@ def test_rejects_bad_arguments_before_any_device_call(lib):
                               1 << 20)) == atf.ATF_ERR_INVALID_ARG  # more keys than slots
     assert _status(lambda: DP(fake, fake, fake, fake, 1, [2], [-1], [100], 8, 28, 4, 128, 1e7, 1.0, fake,
                               1 << 20)) == atf.ATF_ERR_INVALID_ARG  # negative position
+    # distances of 2^31 or more would overflow the kernels' 32-bit windows
+    assert _status(lambda: DP(fake, fake, fake, fake, 1, [4], [5], [5 + (1 << 31)], 8, 28, 4, 128, 1e7,
+                              math.inf, fake, 1 << 20)) == atf.ATF_ERR_UNSUPPORTED
+    assert _status(lambda: DP(fake, fake, fake, fake, 1, [4], [(1 << 32) + 5], [(1 << 32) + 8], 8, 28, 4, 128,
+                              1e7, math.inf, fake, 1)) == atf.ATF_ERR_INVALID_ARG  # far positions pass that check
     assert _status(lambda: atf.atf_decode_merge(fake, 0, 1, 28, 128, fake)) == atf.ATF_ERR_INVALID_ARG
     assert _status(lambda: atf.atf_decode_merge(fake, 2, 1, 28, 96, fake)) == atf.ATF_ERR_UNSUPPORTED
     assert _status(lambda: atf.atf_decode_merge(fake + 4, 2, 1, 28, 128, fake)) == atf.ATF_ERR_INVALID_ARG

@@ -34,6 +34,20 @@ def test_merged_partials_equal_the_decode_oracle(alpha):
         assert np.abs(osk.merge(parts) - want).max() < 1e-12, cuts
 
 
+@pytest.mark.parametrize("alpha", [1.0, math.inf])
+def test_partial_at_far_key_positions_equals_the_near_one(alpha):
+    """Only distances enter the logits: keys rotated at key_pos0 + n with the query
+    at key_pos0 + q_pos give the partial of keys at n with the query at q_pos (up to
+    the fp64 error of angles near 2^31 * omega).  Ignoring key_pos0 would put every
+    key about 2^31 away, outside every finite window."""
+    B, N, Hq, Hkv, d, theta = 1, 400, 4, 2, 64, 1e4
+    q, k, v = _inputs(B, N, Hq, Hkv, d, seed=83)
+    P = (1 << 31) + 12345
+    near = osk.partial(q, oracle.rope(k, theta), v, [0], [N], [N + 6], theta, alpha)
+    far = osk.partial(q, oracle.rope(k, theta, pos0=P), v, [0], [N], [P + N + 6], theta, alpha, key_pos0=[P])
+    assert np.abs(far - near).max() < 1e-5
+
+
 def test_empty_range_merges_as_nothing():
     B, N, Hq, Hkv, d, theta = 1, 64, 2, 1, 64, 1e4
     q, k, v = _inputs(B, N, Hq, Hkv, d, seed=82)

@@ -8,6 +8,7 @@ import pytest
 import torch
 
 import oracle
+from oracle import splitkv as osk
 from rope_frequency_sparse_b200 import atf, splitkv, synth
 
 pytestmark = pytest.mark.gpu
@@ -104,3 +105,28 @@ def test_an_empty_range_contributes_nothing():
     atf.atf_decode_merge(p0, 1, B, Hq, d, b)
     atf.atf_check()
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("alpha", [1.0, math.inf])
+def test_partial_beyond_position_2_31(alpha):
+    """Keys at positions past 2^31 (the query a few positions after the last key):
+    positions are 64-bit, distances stay below 2^31, and with alpha = inf every
+    key keeps every pair (the 32-bit window clamp is exact)."""
+    B, N, Hq, Hkv, d, theta = 1, 3000, 28, 4, 128, 1e7
+    P = (1 << 31) + 12345
+    q = synth.token_major(94, 960, 0, B, 1, Hq, d, torch.bfloat16, threads=1)[:, 0].contiguous()
+    k = synth.token_major(94, 960, 1, B, N, Hkv, d, torch.bfloat16, threads=1)
+    v = synth.token_major(94, 960, 2, B, N, Hkv, d, torch.bfloat16, threads=1)
+    k_rot = torch.from_numpy(oracle.rope(k, theta, pos0=P)).to(torch.bfloat16)  # key n at position P + n
+    _, kc = atf.rope_layout(k_rot.cuda(), 1e4, rotate=False, rotated_out=False, chunked_out=True)
+    q_pos = P + N + 6
+    part = torch.empty(B, Hq, d + 2, dtype=torch.float32, device="cuda")
+    need = atf.atf_decode_workspace_bytes(B, Hq, Hkv, N, d)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    atf.atf_decode_partial(q.cuda(), kc, v.cuda(), part, B, [N], [P], [q_pos], N, Hq, Hkv, d, theta, alpha, ws,
+                           need, None)
+    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device="cuda")
+    atf.atf_decode_merge(part, 1, B, Hq, d, out)
+    atf.atf_check()
+    want = osk.merge(osk.partial(q, k_rot, v, [0], [N], [q_pos], theta, alpha, key_pos0=[P])[None])
+    assert np.abs(out.cpu().double().numpy() - want).max() <= TOL

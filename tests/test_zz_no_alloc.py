@@ -2,9 +2,10 @@
 device memory on the decode path (a host application whose memory manager owns
 all device memory, or a latency-critical loop where an allocation could
 synchronise the device).  Its scratch is a fixed device array inside the
-library; its output must match atf_decode's (which uses a caller workspace)
-within the decode tolerance, on two calls in a row (the second call sees the
-array as the first left it).  Collected last on purpose."""
+library.  It runs the same kernels with the same key-range splits as atf_decode
+(which uses a caller workspace), so its output must be bit-identical to
+atf_decode's, on two calls in a row (the second call sees the array as the first
+left it).  Collected last on purpose."""
 import numpy as np
 import pytest
 import torch
@@ -12,8 +13,6 @@ import torch
 from rope_frequency_sparse_b200 import atf, synth
 
 pytestmark = pytest.mark.gpu
-
-TOL = 2e-2
 
 
 def test_noalloc_decode_matches_workspace_decode_twice():
@@ -31,8 +30,7 @@ def test_noalloc_decode_matches_workspace_decode_twice():
         cnt = torch.zeros(1, dtype=torch.int64, device="cuda")
         atf.atf_decode_noalloc(q, kc, v, out, B, kv_len, N, Hq, Hkv, d, theta, alpha, cnt)
         atf.atf_check()
-        err = (out.float() - ref.float()).abs().max().item()
-        assert err <= TOL, (call, err)
+        assert torch.equal(out, ref), (call, (out.float() - ref.float()).abs().max().item())
         assert int(cnt.item()) == int(cnt_ref.item())
 
 
