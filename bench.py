@@ -1,11 +1,14 @@
 """Benchmark: effective prefill TFLOP/s (and speedup over the same kernel with
-every window open, alpha = inf) on one Qwen2.5-7B-shaped attention layer
-(batch 1, 28 query / 4 kv heads, d = 128, 8192 tokens, bf16, theta = 1e7,
-alpha = 1), plus decode GB/s at a 1,048,576-token cache.
+every window open, alpha = inf) on the largest single-GPU workload: one
+Qwen2.5-7B-shaped attention layer (batch 1, 28 query / 4 kv heads, d = 128,
+theta = 1e7, alpha = 1) of 131072 tokens, prefilled causally in 16 query chunks
+of 8192 against all earlier keys.  The 8k layer with its alpha sweep, the 32k
+pair-energy layer and the 1M-key decode (GB/s) are reported as extra keys.
 
-One step = the whole prefill hot path on one input: RoPE of q and k (fp64
-angles), windowed QK on the tensor cores, online softmax, P.V, epilogue and the
-skipped-pair counter.  Effective FLOPs count only the query-key pairs inside
+One step = the whole prefill hot path on one input: RoPE of k into the cache
+(fp64 angles), then per query chunk RoPE of its queries and the windowed
+prefill (windowed QK on the tensor cores, online softmax, P.V, epilogue, the
+skipped-pair counter).  Effective FLOPs count only the query-key pairs inside
 their window (4 FLOP per active pair) plus P.V (2d FLOP per causal element);
 the exponentials are not counted.
 
@@ -35,22 +38,26 @@ sys.path.insert(0, ROOT)
 
 from rope_frequency_sparse_b200 import atf, synth  # noqa: E402
 
-HEADLINE = "layer_8k"
+HEADLINE = "layer_128k_chunked"
 METRIC = "effective prefill TFLOP/s (alpha=1; active query-key pairs + P.V counted)"
 L2_FLUSH_BYTES = 256 << 20
 
 
 # ------------------------------------------------------------------ accounting (host integers)
 
-def window_table(d, theta, alpha):
-    return [int(w) for w in atf.atf_windows(d, theta, alpha)]
+def window_table(d, theta, alpha, windows=None):
+    """W_i as Python ints: from the library (our arm) or from `windows` (the
+    reference arm passes the oracle's table, so that arm loads no CUDA code)."""
+    if windows is not None:
+        return [int(x) for x in windows(d, theta, alpha)]
+    return [int(x) for x in atf.atf_windows(d, theta, alpha)]
 
 
-def prefill_flops(w: synth.Workload, alpha: float, seq: int | None = None) -> tuple[int, int, int]:
+def prefill_flops(w: synth.Workload, alpha: float, seq: int | None = None, windows=None) -> tuple[int, int, int]:
     """(effective FLOPs, dense FLOPs, skipped pairs) of a causal prefill over `seq` tokens."""
     S = w.seq if seq is None else seq
     P = S * (S + 1) // 2
-    W = window_table(w.d, w.theta, alpha)
+    W = window_table(w.d, w.theta, alpha, windows)
     skipped = sum((S - 1 - x) * (S - x) // 2 for x in W if x < S - 1)
     active = (w.d // 2) * P - skipped
     eff = w.batch * w.q_heads * (4 * active + 2 * w.d * P)
@@ -58,10 +65,16 @@ def prefill_flops(w: synth.Workload, alpha: float, seq: int | None = None) -> tu
     return eff, dense, w.q_heads * skipped * w.batch
 
 
-def row_flops(w: synth.Workload, alpha: float, m: int) -> int:
-    W = window_table(w.d, w.theta, alpha)
+def row_flops(w: synth.Workload, alpha: float, m: int, windows=None) -> int:
+    W = window_table(w.d, w.theta, alpha, windows)
     active = sum(min(m, x) + 1 for x in W)  # pairs i with (m - n) <= W_i over n = 0..m
     return 4 * active + 2 * w.d * (m + 1)
+
+
+def causal_elements(w: synth.Workload, seq: int | None = None) -> int:
+    """Query-key elements (m, n <= m) of the prefill, all heads: one exponential each."""
+    S = w.seq if seq is None else seq
+    return w.batch * w.q_heads * S * (S + 1) // 2
 
 
 def decode_bytes(w: synth.Workload, alpha: float) -> tuple[int, int]:
@@ -191,6 +204,57 @@ class PrefillStep:
             ev[2].record(stream)
 
 
+class ChunkedPrefillStep:
+    """Device-resident inputs and scratch for the chunked prefill of a long layer:
+    keys rotated once into a cache, then per query chunk its queries rotated at
+    their offset and attended against all earlier keys."""
+
+    def __init__(self, w: synth.Workload, seed: int, device):
+        q, k, v = synth.prefill_inputs(w, seed=seed)
+        self.w = w
+        self.host = (q, k, v)
+        self.q, self.k, self.v = q.to(device), k.to(device), v.to(device)
+        B, S, Hq, d = self.q.shape
+        self.k_rot = torch.empty_like(self.k)
+        self.q_rot = torch.empty((B, w.q_chunk, Hq, d), dtype=self.q.dtype, device=device)
+        self.out = torch.empty_like(self.q)
+        self.cnt = torch.zeros(1, dtype=torch.int64, device=device)
+        self.n_chunks = S // w.q_chunk
+
+    def n_events(self):
+        return 2 + 2 * self.n_chunks
+
+    def run(self, alpha, stream, ev=None, count=True):
+        """RoPE k, then per chunk RoPE q + windowed prefill: 1 + 2 x chunks launches.
+        ev = (step start, step end, then start/end of each chunk's prefill kernel)."""
+        w = self.w
+        B, S, Hq, d = self.q.shape
+        Hkv = self.k.shape[2]
+        C = w.q_chunk
+        if ev:
+            ev[0].record(stream)
+        atf.atf_rope_layout(self.k, self.k_rot, None, B, S, Hkv, d, 0, w.theta, 1, atf.ATF_BF16, stream)
+        for c in range(self.n_chunks):
+            c0 = c * C
+            atf.atf_rope_layout(self.q[:, c0:c0 + C], self.q_rot, None, B, C, Hq, d, c0, w.theta, 1, atf.ATF_BF16,
+                                stream)
+            if ev:
+                ev[2 + 2 * c].record(stream)
+            atf.atf_prefill_ex(self.q_rot, self.k_rot, self.v, self.out[:, c0:c0 + C], B, C, c0 + C, Hq, Hkv, d, c0,
+                               atf.ATF_BF16, 1, w.theta, alpha, self.cnt if count else None, None, 0, stream)
+            if ev:
+                ev[3 + 2 * c].record(stream)
+        if ev:
+            ev[1].record(stream)
+
+    @staticmethod
+    def times(evs):
+        """(mean ms per step, mean ms of the prefill kernels per step) of timed steps."""
+        step = [e[0].elapsed_time(e[1]) for e in evs]
+        kern = [sum(e[2 + 2 * c].elapsed_time(e[3 + 2 * c]) for c in range((len(e) - 2) // 2)) for e in evs]
+        return sum(step) / len(step), sum(kern) / len(kern)
+
+
 def time_steps(fn, steps, warmup, stream, flush_buf, n_events=3):
     """Run warmup + steps; per-step CUDA events (the L2 flush between steps is
     outside the events).  Returns list of per-step event-lists."""
@@ -202,6 +266,24 @@ def time_steps(fn, steps, warmup, stream, flush_buf, n_events=3):
     for i in range(steps):
         flush_l2(flush_buf)
         fn(evs[i])
+    torch.cuda.synchronize()
+    return evs
+
+
+def time_interleaved(fns, steps, warmup, stream, flush_buf, n_events):
+    """Warm up every step function, then run `steps` rounds of all of them in turn,
+    so that they see the same clocks and power state; per-step CUDA events (the L2
+    flush between steps outside them).  Returns one list of event-lists per fn."""
+    for _ in range(warmup):
+        for fn in fns:
+            flush_l2(flush_buf)
+            fn(None)
+    torch.cuda.synchronize()
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(n_events)] for _ in range(steps)] for _ in fns]
+    for i in range(steps):
+        for f, fn in enumerate(fns):
+            flush_l2(flush_buf)
+            fn(evs[f][i])
     torch.cuda.synchronize()
     return evs
 
@@ -221,14 +303,17 @@ def barrier():
 
 # ------------------------------------------------------------------ CPU oracle baseline
 
-def cpu_oracle_sample(w: synth.Workload, alpha: float, target_s: float = 12.0, seed=synth.DEFAULT_SEED):
-    """Time the fp64 oracle on a bounded sample of query rows of the workload."""
+def cpu_oracle_sample(w: synth.Workload, alpha: float, target_s: float = 12.0, seed=synth.DEFAULT_SEED,
+                      inputs=None):
+    """Time the fp64 oracle on a bounded sample of query rows of the workload (the
+    rows of a chunked workload are the same rows of the unchunked prefill)."""
     import oracle  # test infrastructure: the CPU baseline only
 
-    q, k, v = synth.prefill_inputs(w, seed=seed)
+    win = lambda d, theta, a: oracle.windows(d, theta, a)[0]  # noqa: E731
+    q, k, v = inputs if inputs is not None else synth.prefill_inputs(w, seed=seed)
     cores = os.cpu_count() or 1
     rng = np.random.default_rng(0)
-    n_rows = 8
+    n_rows = 2
     while True:
         rows = np.sort(rng.choice(w.seq, size=n_rows, replace=False))
         t0 = time.perf_counter()
@@ -237,34 +322,42 @@ def cpu_oracle_sample(w: synth.Workload, alpha: float, target_s: float = 12.0, s
         if dt >= target_s or n_rows >= w.seq:
             break
         n_rows = min(w.seq, max(n_rows * 2, int(n_rows * target_s / max(dt, 1e-3))))
-    flops = w.batch * w.q_heads * sum(row_flops(w, alpha, int(m)) for m in rows)
+    flops = w.batch * w.q_heads * sum(row_flops(w, alpha, int(m), win) for m in rows)
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{len(rows)} random query rows x {w.q_heads} heads of {w.name} (alpha={alpha}); "
-                      f"{dt:.1f} s wall; includes the oracle's one-time fp64 rotation of all keys",
+            "sample": f"{len(rows)} random query rows x {w.q_heads} heads of {w.name} (alpha={alpha}), each "
+                      f"against all its earlier keys; {dt:.1f} s wall; includes the oracle's one-time fp64 "
+                      "rotation of all keys",
             "seconds": dt}
 
 
 # ------------------------------------------------------------------ arms
 
+def headline_config(w: synth.Workload, world: int) -> dict:
+    return {"workload": w.name, "batch": w.batch, "seq_len": w.seq, "query_chunk": w.q_chunk,
+            "q_heads": w.q_heads, "kv_heads": w.kv_heads, "d": w.d, "theta": w.theta, "alpha": 1.0,
+            "parallelism": f"independent layers x{world}",
+            "l2": "inputs (1.2 GB) larger than L2, and a 256 MiB write between steps outside the CUDA events"}
+
+
 def run_reference(args, rank):
-    """The fp64 CPU oracle as it stands, on this arm's workload and metric."""
+    """The fp64 CPU oracle as it stands, on this arm's workload and metric (no
+    CUDA code is loaded: FLOPs are counted with the oracle's own window table)."""
     if rank != 0:
         return
     w = synth.WORKLOADS[HEADLINE]
-    vals = []
+    inputs = synth.prefill_inputs(w)
     for _ in range(args.warmup):
-        cpu_oracle_sample(w, 1.0, target_s=2.0)
-    samples = []
+        cpu_oracle_sample(w, 1.0, target_s=2.0, inputs=inputs)
+    vals, samples = [], []
     for _ in range(args.steps):
-        s = cpu_oracle_sample(w, 1.0, target_s=6.0)
-        vals.append(s["value"])
-        samples.append(s)
+        smp = cpu_oracle_sample(w, 1.0, target_s=5.0, inputs=inputs)
+        vals.append(smp["value"])
+        samples.append(smp)
     v = statistics.median(vals)
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64)",
-            "config": {"workload": HEADLINE, "batch": 1, "seq_len": w.seq, "q_heads": 28, "kv_heads": 4, "d": 128,
-                       "theta": w.theta, "alpha": 1.0},
+            "config": headline_config(w, 1),
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": samples[-1]["cores"], "kind": "oracle",
                              "sample": samples[-1]["sample"]},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -276,47 +369,53 @@ def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream()
+    s = stream
     peaks, peak_kind = measured_peaks()
+    n_sm = torch.cuda.get_device_properties(device).multi_processor_count
     w = synth.WORKLOADS[HEADLINE]
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-    step = PrefillStep(w, synth.DEFAULT_SEED + rank, device)
-    s = stream
+    step = ChunkedPrefillStep(w, synth.DEFAULT_SEED + rank, device)
+    nev = step.n_events()
 
     # ---- headline: alpha = 1, timed region bracketed by barrier + sync
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clocks:
         t_wall = time.perf_counter()
-        evs = time_steps(lambda ev: step.run(1.0, s, ev), args.steps, args.warmup, stream, flush_buf)
+        evs = time_steps(lambda ev: step.run(1.0, s, ev), args.steps, args.warmup, stream, flush_buf, n_events=nev)
         t_wall = time.perf_counter() - t_wall
     barrier()
     torch.cuda.synchronize()
     atf.atf_check(s)
-    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
-    kern_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    ms_step = dist_max(sum(step_ms) / len(step_ms))
-    ms_kern = dist_max(sum(kern_ms) / len(kern_ms))
+    ms_step, ms_kern = ChunkedPrefillStep.times(evs)
+    ms_step, ms_kern = dist_max(ms_step), dist_max(ms_kern)
     eff, dense_flops, skipped = prefill_flops(w, 1.0)
     value = world * eff / (ms_step * 1e-3) / 1e12
     cnt_per_step = int(step.cnt.item()) // (args.steps + args.warmup)
 
-    # ---- the same step with every window open (the dense specialisation)
-    evs_d = time_steps(lambda ev: step.run(math.inf, s, ev), args.steps, args.warmup, stream, flush_buf)
-    ms_dense = dist_max(sum(e[0].elapsed_time(e[2]) for e in evs_d) / args.steps)
-    ms_dense_kern = dist_max(sum(e[1].elapsed_time(e[2]) for e in evs_d) / args.steps)
-    per_alpha = {}
-    for a in w.alphas:
-        if a in (1.0,) or math.isinf(a):
-            continue
-        ev_a = time_steps(lambda ev: step.run(a, s, ev), max(3, args.steps // 2), 1, stream, flush_buf)
-        ms_a = sum(e[0].elapsed_time(e[2]) for e in ev_a) / len(ev_a)
-        per_alpha[str(a)] = {"tflops": prefill_flops(w, a)[0] / (ms_a * 1e-3) / 1e12, "ms": ms_a}
-    per_alpha["1.0"] = {"tflops": eff / (ms_step * 1e-3) / 1e12, "ms": ms_step}
-    per_alpha["inf"] = {"tflops": dense_flops / (ms_dense * 1e-3) / 1e12, "ms": ms_dense}
+    # ---- the same step with every window open (the dense specialisation) and with
+    # alpha = 0.5, interleaved step by step with alpha = 1 so that all three see the
+    # same clocks: the windowed kernel draws less power and keeps higher clocks under
+    # the power cap, which a back-to-back comparison would credit to the method
+    with ClockSampler(local_rank) as clocks_i:
+        ev_i = time_interleaved([lambda ev: step.run(1.0, s, ev, count=False),
+                                 lambda ev: step.run(math.inf, s, ev, count=False),
+                                 lambda ev: step.run(0.5, s, ev, count=False)],
+                                max(3, args.steps // 2), args.warmup, stream, flush_buf, nev)
+    (ms_one, ms_one_kern), (ms_dense, ms_dense_kern), (ms_half, ms_half_kern) = (
+        tuple(dist_max(x) for x in ChunkedPrefillStep.times(e)) for e in ev_i)
+    eff_half = prefill_flops(w, 0.5)[0]
+    per_alpha = {"0.5": {"tflops": eff_half / (ms_half * 1e-3) / 1e12, "ms": ms_half, "kernel_ms": ms_half_kern,
+                         "speedup_vs_dense": ms_dense / ms_half},
+                 "1.0": {"tflops": eff / (ms_one * 1e-3) / 1e12, "ms": ms_one, "kernel_ms": ms_one_kern,
+                         "speedup_vs_dense": ms_dense / ms_one},
+                 "inf": {"tflops": dense_flops / (ms_dense * 1e-3) / 1e12, "ms": ms_dense, "kernel_ms": ms_dense_kern},
+                 "note": "the three steps interleaved (one of each per round), clocks in clocks_interleaved"}
 
     # ---- end to end through the C ABI from pinned host buffers: atf_prefill_host
-    # uploads q, k, v, runs RoPE + the windowed prefill and downloads the output,
-    # the copies overlapped with each other and with the kernels
+    # uploads q, k, v, rotates and attends query chunks of 8192 rows as they land,
+    # and downloads each chunk's output, copies overlapped with each other and with
+    # the kernels
     q_h, k_h, v_h = (t.pin_memory() for t in step.host)
     out_h = torch.empty_like(q_h).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
@@ -324,54 +423,63 @@ def run_ours(args, rank, world, local_rank):
     B, S, Hq, d = step.q.shape
     Hkv = step.k.shape[2]
     hws_bytes = atf.atf_prefill_host_workspace_bytes(B, S, S, Hq, Hkv, d, 0)
+    del step.out
+    torch.cuda.empty_cache()
     hws = torch.empty(hws_bytes, dtype=torch.uint8, device=device)
 
-    def e2e_step(ev, chunk_rows=0):
+    def e2e_step(ev):
         if ev:
             ev[0].record(stream)
         atf.atf_prefill_host(q_h, k_h, v_h, out_h, B, S, S, Hq, Hkv, d, 0, 0, w.theta, 1.0, hws, hws_bytes,
-                             chunk_rows, None, s)
+                             w.q_chunk, None, s)
         if ev:
             ev[1].record(stream)
 
-    evs_e = time_steps(e2e_step, args.steps, args.warmup, stream, flush_buf, n_events=2)
-    ms_e2e = dist_max(sum(e[0].elapsed_time(e[1]) for e in evs_e) / args.steps)
+    evs_e = time_steps(e2e_step, min(args.steps, 5), args.warmup, stream, flush_buf, n_events=2)
+    ms_e2e = dist_max(sum(e[0].elapsed_time(e[1]) for e in evs_e) / len(evs_e))
     e2e_val = world * eff / (ms_e2e * 1e-3) / 1e12
     atf.atf_check(s)
-    e2e_sweep = {}
-    if world == 1 and not args.no_extra:
-        for rows in (512, 1024, 2048, S):
-            ev_c = time_steps(lambda ev: e2e_step(ev, rows), max(3, args.steps // 2), 1, stream, flush_buf,
-                              n_events=2)
-            e2e_sweep[str(rows)] = sum(e[0].elapsed_time(e[1]) for e in ev_c) / len(ev_c)
+    del hws, step
+    torch.cuda.empty_cache()
 
     extra = {}
     if world == 1 and not args.no_extra:
         extra = run_extra(args, device, stream, flush_buf, peaks)
 
+    ck = clocks.summary()
+    sm_mhz = ck.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
     tflops_kern = eff / (ms_kern * 1e-3) / 1e12
-    traffic = recorded_traffic("prefill_tc.cu", "prefill_tc_layer_8k.md")
+    exps = causal_elements(w)
+    ex2_rate = exps / (ms_kern * 1e-3)
+    ex2_peak = 16 * n_sm * sm_mhz * 1e6
+    traffic = recorded_traffic("prefill_tc.cu", "prefill_tc_layer_128k_chunk.md")
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded numpy PCG64 N(0,1) -> bf16)",
-        "config": {"workload": HEADLINE, "batch": 1, "seq_len": w.seq, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
-                   "d": w.d, "theta": w.theta, "alpha": 1.0, "parallelism": f"independent layers x{world}",
-                   "l2": "flushed between steps (256 MiB write, outside the per-step CUDA events)"},
-        "speedup_vs_dense": ms_dense / ms_step,
-        "kernel_speedup_vs_dense": ms_dense_kern / ms_kern,
+        "config": headline_config(w, world),
+        "speedup_vs_dense": ms_dense / ms_one,
+        "kernel_speedup_vs_dense": ms_dense_kern / ms_one_kern,
         "per_alpha": per_alpha,
         "skipped_pairs_per_step": cnt_per_step, "skipped_pairs_closed_form": skipped,
         "roofline": {"bound": "tensor", "achieved": tflops_kern, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": tflops_kern / peaks["bf16_tflops"], "traffic": traffic,
-                     "kernel": "prefill_tc_kernel<128,sparse>", "peak_kind": f"{peak_kind} bf16 burst",
-                     "kernel_ms": ms_kern},
+                     "kernel": "prefill_tc_kernel<128,sparse>, 16 launches per step", "kernel_ms": ms_kern,
+                     "peak_kind": f"{peak_kind} bf16 burst",
+                     "peak_sustained": peaks.get("bf16_tflops_sustained"),
+                     "frac_sustained": tflops_kern / peaks["bf16_tflops_sustained"]
+                     if peaks.get("bf16_tflops_sustained") else None,
+                     "dense_kernel_tflops": dense_flops / (ms_dense_kern * 1e-3) / 1e12},
+        "sfu_ex2_roof": {"exponentials_per_step": exps, "achieved_per_s": ex2_rate, "peak_per_s": ex2_peak,
+                         "frac": ex2_rate / ex2_peak, "sm_mhz": sm_mhz,
+                         "peak_basis": f"16 ex2 per clock per SM (measured) x {n_sm} SMs x the median SM clock "
+                                       "sampled during the timed steps"},
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": ms_e2e,
-                "call": "atf_prefill_host (pinned host buffers, default chunk schedule, two compute streams)",
-                "ms_by_chunk_rows": e2e_sweep},
-        "gpu_launches": 3 * args.steps,  # rope(q), rope(k), prefill per step of the device-resident timing
-        "clocks": clocks.summary(),
+                "call": "atf_prefill_host (pinned host buffers, query chunks of 8192 rows, two copy streams)"},
+        "gpu_launches": (1 + 2 * (w.seq // w.q_chunk)) * args.steps,  # rope(k), then rope(q) + prefill per chunk
+        "clocks": ck,
+        "clocks_interleaved": clocks_i.summary(),
         "wall_s_timed_region": t_wall,
     }
     line.update(extra)
@@ -382,19 +490,32 @@ def run_ours(args, rank, world, local_rank):
 
 
 def run_extra(args, device, stream, flush_buf, peaks):
-    """Secondary workloads: the 8k step with rotate-half pairs, 32k pair-energy
-    prefill, 128k chunked prefill, 1M-key decode."""
+    """Secondary workloads: the 8k layer (alpha sweep against the dense kernel,
+    and rotate-half pairs), 32k pair-energy prefill, 1M-key decode, split-KV
+    decode, FASA-style decode, KV-cache append."""
     s = stream
     out = {}
-    # the headline 8k step with q, k read as rotate-half (NeoX-style) pairs
-    w2 = synth.WORKLOADS[HEADLINE]
-    st2 = PrefillStep(w2, synth.DEFAULT_SEED, device)
-    ev2 = time_steps(lambda ev: st2.run(1.0, s, ev, pairing=atf.ATF_PAIRS_ROTATE_HALF), 5, 3, stream, flush_buf)
+    # the 8k layer: alpha sweep, each against the same step with every window open
+    w8 = synth.WORKLOADS["layer_8k"]
+    st8 = PrefillStep(w8, synth.DEFAULT_SEED, device)
+    res8 = {}
+    for a in w8.alphas:
+        ev8 = time_steps(lambda ev: st8.run(a, s, ev), 10, 3, stream, flush_buf)
+        ms8 = sum(e[0].elapsed_time(e[2]) for e in ev8) / len(ev8)
+        ms8k = sum(e[1].elapsed_time(e[2]) for e in ev8) / len(ev8)
+        f8 = prefill_flops(w8, a)[0] if not math.isinf(a) else prefill_flops(w8, a)[1]
+        res8[str(a)] = {"tflops": f8 / (ms8 * 1e-3) / 1e12, "ms": ms8, "kernel_ms": ms8k,
+                        "kernel_tflops": f8 / (ms8k * 1e-3) / 1e12}
+    res8["speedup_vs_dense_alpha1"] = res8["inf"]["ms"] / res8["1.0"]["ms"]
+    res8["kernel_speedup_vs_dense_alpha1"] = res8["inf"]["kernel_ms"] / res8["1.0"]["kernel_ms"]
+    res8["kernel_frac_of_peak_alpha1"] = res8["1.0"]["kernel_tflops"] / peaks["bf16_tflops"]
+    ev2 = time_steps(lambda ev: st8.run(1.0, s, ev, pairing=atf.ATF_PAIRS_ROTATE_HALF), 5, 3, stream, flush_buf)
     ms2 = sum(e[0].elapsed_time(e[2]) for e in ev2) / 5
     ms2r = sum(e[0].elapsed_time(e[1]) for e in ev2) / 5
-    eff2 = prefill_flops(w2, 1.0)[0]
-    out["layer_8k_rotate_half"] = {"tflops": eff2 / (ms2 * 1e-3) / 1e12, "ms": ms2, "rope_ms": ms2r}
-    del st2
+    res8["rotate_half_alpha1"] = {"tflops": prefill_flops(w8, 1.0)[0] / (ms2 * 1e-3) / 1e12, "ms": ms2,
+                                  "rope_ms": ms2r}
+    out["layer_8k"] = res8
+    del st8
     torch.cuda.empty_cache()
     # 32k tokens, pair-energy-scaled q/k
     w3 = synth.WORKLOADS["layer_32k_pair_energy"]
@@ -409,40 +530,6 @@ def run_extra(args, device, stream, flush_buf, peaks):
                                     "kernel_frac_of_peak": eff3 / (ms3k * 1e-3) / 1e12 / peaks["bf16_tflops"],
                                     "speedup_vs_dense": ms3d / ms3}
     del st3
-    torch.cuda.empty_cache()
-
-    # 131072 tokens in 16 query chunks of 8192 (keys rotated once into the cache)
-    w4 = synth.WORKLOADS["layer_128k_chunked"]
-    q, k, v = synth.prefill_inputs(w4)
-    qd, kd, vd = q.to(device), k.to(device), v.to(device)
-    del q, k, v
-    B, S, Hq, d = qd.shape
-    Hkv = kd.shape[2]
-    k_rot = torch.empty_like(kd)
-    q_rot = torch.empty((B, w4.q_chunk, Hq, d), dtype=qd.dtype, device=device)
-    o4 = torch.empty_like(qd)
-    C = w4.q_chunk
-
-    def chunked(alpha, ev):
-        if ev:
-            ev[0].record(stream)
-        atf.atf_rope_layout(kd, k_rot, None, B, S, Hkv, d, 0, w4.theta, 1, atf.ATF_BF16, s)
-        for c0 in range(0, S, C):
-            atf.atf_rope_layout(qd[:, c0:c0 + C], q_rot, None, B, C, Hq, d, c0, w4.theta, 1, atf.ATF_BF16, s)
-            atf.atf_prefill_ex(q_rot, k_rot, vd, o4[:, c0:c0 + C], B, C, c0 + C, Hq, Hkv, d, c0, atf.ATF_BF16, 1,
-                               w4.theta, alpha, None, None, 0, s)
-        if ev:
-            ev[1].record(stream)
-
-    res4 = {}
-    for a in (1.0, 0.5, math.inf):
-        ev4 = time_steps(lambda ev: chunked(a, ev), 2, 1, stream, flush_buf, n_events=2)
-        ms4 = sum(e[0].elapsed_time(e[1]) for e in ev4) / 2
-        f4 = prefill_flops(w4, a)[0] if not math.isinf(a) else prefill_flops(w4, a)[1]
-        res4[str(a)] = {"tflops": f4 / (ms4 * 1e-3) / 1e12, "ms": ms4}
-    res4["speedup_vs_dense_alpha1"] = res4["inf"]["ms"] / res4["1.0"]["ms"]
-    out["layer_128k_chunked"] = res4
-    del qd, kd, vd, k_rot, q_rot, o4
     torch.cuda.empty_cache()
 
     # decode: 4 sequences x 1,048,576 cached keys (device-generated seeded normals)
@@ -585,6 +672,39 @@ def run_extra(args, device, stream, flush_buf, peaks):
     return out
 
 
+def run_chunk_profile(args):
+    """Only the last query chunk of the 131072-token layer (the heaviest launch of
+    the headline step): ROWS query rows ending at position 131071 against all
+    131072 keys, windowed (alpha = 1) then dense, W + K prefill launches each, for
+    ncu captures.  Inputs are seeded device normals of the workload's shapes."""
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    w = synth.WORKLOADS[HEADLINE]
+    S, C = w.seq, args.profile_chunk
+    g = torch.Generator(device=device)
+    g.manual_seed(synth.DEFAULT_SEED)
+    q = torch.randn((1, C, w.q_heads, w.d), generator=g, device=device).to(torch.bfloat16)
+    k = torch.randn((1, S, w.kv_heads, w.d), generator=g, device=device).to(torch.bfloat16)
+    v = torch.randn((1, S, w.kv_heads, w.d), generator=g, device=device).to(torch.bfloat16)
+    s = torch.cuda.current_stream()
+    q_rot, k_rot, out = torch.empty_like(q), torch.empty_like(k), torch.empty_like(q)
+    atf.atf_rope_layout(k, k_rot, None, 1, S, w.kv_heads, w.d, 0, w.theta, 1, atf.ATF_BF16, s)
+    atf.atf_rope_layout(q, q_rot, None, 1, C, w.q_heads, w.d, S - C, w.theta, 1, atf.ATF_BF16, s)
+    res = {}
+    for alpha in (1.0, math.inf):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for it in range(args.warmup + args.steps):
+            if it == args.warmup:
+                e0.record(s)
+            atf.atf_prefill_ex(q_rot, k_rot, v, out, 1, C, S, w.q_heads, w.kv_heads, w.d, S - C, atf.ATF_BF16, 1,
+                               w.theta, alpha, None, None, 0, s)
+        e1.record(s)
+        atf.atf_check(s)
+        res[str(alpha)] = e0.elapsed_time(e1) / max(args.steps, 1)
+    print(json.dumps({"profile": "prefill_chunk", "query_rows": C, "keys": S, "launches_per_alpha":
+                      args.warmup + args.steps, "ms_per_launch": res}))
+
+
 def run_decode_profile(args):
     """Only the decode step (alpha = 1) with a shortened cache, for ncu captures:
     the decode_1m shapes with KEYS cached keys per sequence, W + K launches."""
@@ -654,12 +774,17 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--profile-decode", type=int, metavar="KEYS", default=0,
                     help="run only the decode step with KEYS cached keys per sequence (for ncu captures)")
+    ap.add_argument("--profile-chunk", type=int, metavar="ROWS", default=0,
+                    help="run only the last ROWS query rows of the 131072-token layer (for ncu captures)")
     ap.add_argument("--profile-fasa", type=int, metavar="KEYS", default=0,
                     help="run only the FASA-style decode on one sequence of KEYS keys (for ncu captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.profile_decode:
         run_decode_profile(args)
+        return
+    if args.profile_chunk:
+        run_chunk_profile(args)
         return
     if args.profile_fasa:
         run_fasa_profile(args)

@@ -13,7 +13,9 @@
 // every K and V tile; 12 warps in three warpgroups:
 //   warp 0      TMA producer: both Q~ tiles once, then K and V tiles of 128 keys
 //               (128B-swizzled boxes of 64 dims) into separate rings.
-//   warp 1      TMEM owner and MMA issuer (one thread), per KV tile j and Q tile g:
+//   warp 1      TMEM owner and MMA issuer: the warp runs its loop convergently
+//               and one elected lane issues the MMAs and commits; per KV tile j
+//               and Q tile g:
 //                 S_g(j)  = Q~_g . K~(j)^T      A = Q~_g (smem), B = K tile (smem)
 //                 O_g    += P_g(j) . V(j)       A = P_g in TMEM, B = V tile (MN-major)
 //   warps 2-3   idle (they complete warpgroup 0 for the register reallocation)
@@ -22,7 +24,7 @@
 // Warpgroup 0 gives registers to the two softmax warpgroups (setmaxnreg), so a
 // thread holds its whole 128-column row of S at once.
 // TMEM columns: S_g at [128 g, 128 g + 128) (P_g written back over it as packed
-// bf16), O_g at [256 + g d, 256 + (g + 1) d).
+// bf16, in two pieces of 64 keys), O_g at [256 + g d, 256 + (g + 1) d).
 // Issue order: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ... so one Q tile's
 // exponentials overlap the other tile's MMAs.
 //
@@ -39,6 +41,11 @@
 // subtracted; only straddling pairs, and only 32-column chunks a warp's rows
 // reach, are touched.  The window counts come from the W table held across each
 // warp's lanes (ballots), with no per-tile table.
+// The softmax loop has two bodies.  The correcting body runs only on the tiles
+// where a window boundary crosses the warp's elements or where pairs die at the
+// next tile; between those, runs of clean tiles (every pair dead or live for
+// all of the warp's elements) go through a body that is the dense kernel's loop
+// plus one counter update, with none of the correction code in it.
 //
 // Exponentials.  The SFU evaluates 16 ex2 per clock per SM, as many as the
 // tensor core needs cycles for a 128x128 tile's two MMAs.  A share of the column
@@ -48,6 +55,7 @@
 #include <cuda_bf16.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "atf_internal.cuh"
 #include "ptx.cuh"
@@ -90,7 +98,7 @@ struct Cfg {
 };
 
 struct Shared {
-  uint64_t q_full[NQ], q_ready[NQ], s_full[NQ], p_half[NQ], p_full[NQ], o_done[NQ];
+  uint64_t q_full[NQ], q_ready[NQ], s_full[NQ], p_bar[NQ][2], o_done[NQ];
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint64_t drain;
   uint32_t tmem_base;
@@ -129,6 +137,10 @@ struct WarpWindows {
   // number of pairs with W_i < x (W is non-decreasing); warp-collective
   __device__ __forceinline__ int below(long long x) const {
     return __popc(__ballot_sync(0xffffffffu, w0 < x)) + __popc(__ballot_sync(0xffffffffu, w1 < x));
+  }
+  // W_i (i warp-uniform, i < 64); warp-collective
+  __device__ __forceinline__ long long at(int i) const {
+    return __shfl_sync(0xffffffffu, i < 32 ? w0 : w1, i & 31);
   }
   __device__ __forceinline__ uint32_t quarter_ranges(long long center, int q) const {
     const long long lo = center + 32 * q;
@@ -222,6 +234,10 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
 #endif
 __host__ __device__ constexpr bool exp_on_fma(int k) { return (ATF_EXP_FMA_MASK >> (k & 7)) & 1; }
 
+// P goes to the MMA warp in two pieces of 64 keys (the P.V of the first runs while
+// the softmax computes the second).
+constexpr int kPPieces = 2;
+
 }  // namespace
 
 template <int D, bool SPARSE>
@@ -269,8 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh->q_full[g], 1);
       mbar_init(&sh->q_ready[g], 128);
       mbar_init(&sh->s_full[g], 1);
-      mbar_init(&sh->p_half[g], 128);
-      mbar_init(&sh->p_full[g], 128);
+      for (int pc = 0; pc < 2; ++pc) mbar_init(&sh->p_bar[g][pc], 128);
       mbar_init(&sh->o_done[g], 1);
     }
     for (int s = 0; s < NSK; ++s) {
@@ -354,7 +369,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int g = 0; ok && g < nq; ++g) ok = warp_wait(&sh->q_ready[g], 0, abort, p.err, 0x201);
       tc_fence_after();
-      int k_seen = 0;  // K tiles whose arrival this thread has observed
+      int k_seen = 0;  // K tiles whose arrival this warp has observed
+      // S_g(j) = Q~_g . K(j)^T over the active 8-pair chunks
       auto issue_s = [&](int g, int j) -> bool {
         const int s = j % NSK;
         if (j >= k_seen) {
@@ -395,19 +411,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t o_tmem = tmem + C::COL_O + g * D;
             const uint64_t bv = dv0 + sv * kTileStep;
             const bool first = j == jstart(g);
-            // P arrives in two halves (keys 0..63, then 64..127): the first half's
-            // P.V runs while the softmax still computes the second
+            // P arrives in kPPieces pieces of BN / kPPieces keys: the P.V of a piece
+            // runs while the softmax still computes the later ones
+            constexpr int KK = BN / 16 / kPPieces;  // K-steps (16 keys) per piece
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              if (!(ok = warp_wait(half ? &sh->p_full[g] : &sh->p_half[g], (j - jstart(g)) & 1, abort, p.err,
-                                   0x204 + half)))
-                break;
+            for (int pc = 0; pc < kPPieces; ++pc) {
+              if (!(ok = warp_wait(&sh->p_bar[g][pc], (j - jstart(g)) & 1, abort, p.err, 0x210 + pc))) break;
               tc_fence_after();
               if (elect_one()) {
 #pragma unroll
-                for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
+                for (int kk = KK * pc; kk < KK * pc + KK; ++kk)
                   mma_ts(o_tmem, p_tmem + 8 * kk, bv + ((kk * 2048) >> 4), idesc_pv, (!first || kk > 0) ? 1u : 0u);
-                if (half && j == T - 1) mma_commit(&sh->o_done[g]);
+                if (pc == kPPieces - 1 && j == T - 1) mma_commit(&sh->o_done[g]);
               }
               __syncwarp();
             }
@@ -471,33 +486,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t lsum2 = 0ull;  // packed partial row sums
       unsigned long long cnt = 0;
       int zst = 0;  // first pair held in this warp's rows of the stash
-      uint32_t qr = SPARSE ? ww.quarter_ranges(centre(j0 + g), quarter) : 0u;
-      for (int j = j0; ok && j < T; ++j) {
+
+      // The softmax of one KV tile j.  CORR = true: the correcting body, for tiles
+      // on which a window boundary crosses this warp's rows (straddling pairs are
+      // added back or subtracted on S) or after which pairs die (zeroed in Q~);
+      // CORR = false: the clean body, on which every pair is dead for all of this
+      // warp's elements (the first a_run pairs) or live for all of them -- the
+      // dense kernel's loop plus one counter update.
+      auto tile = [&](const int j, auto corr_tag, const int a_run) -> bool {
+        constexpr bool CORR = decltype(corr_tag)::value;
         const int s = j % NSK;
         const long long n0 = tile_n0(j);
         const long long center = m0 + g * BM - n0;
-        const int z = static_cast<int>(qr & 0xFF);
-        const int a = static_cast<int>((qr >> 8) & 0xFF);
-        const int u = static_cast<int>((qr >> 16) & 0xFF);
-        // the next tile's ranges, computed while S is still on its way
-        const uint32_t qr_next = (SPARSE && j + 1 < T) ? ww.quarter_ranges(center + BN, quarter) : 0u;
         // valid columns of this row form the prefix [0, cmax]
         int cmax = -1;
         if (row_ok) cmax = static_cast<int>(min(static_cast<long long>(BN - 1), min(m, kv_last) - n0));
         const bool partial = __any_sync(0xffffffffu, cmax < BN - 1);
-        // (everything up to the wait is independent of S, off the softmax -> MMA chain)
-        // no S MMA when every pair is zeroed in every row
-        const bool has_mma = !SPARSE || (ww.below(center + kZeroOffset) >> 3) < C::NCH;
         const int nv = cmax + 1;  // valid columns of this row
-        if (SPARSE) cnt += static_cast<unsigned long long>(a) * nv;
-        const int cmax_w = (SPARSE && a < u) ? __reduce_max_sync(0xffffffffu, cmax) : 0;
+        if constexpr (SPARSE && !CORR) cnt += static_cast<unsigned long long>(a_run) * nv;
+        // (everything up to the wait is independent of S, off the softmax -> MMA chain)
+        uint32_t qr = 0u, qr_next = 0u;
+        int z = 0, a = 0, u = 0, cmax_w = 0, cw = 0, wl0 = 0;
+        bool has_mma = true;
+        uint32_t tb0[BN / 32] = {}, fb0[BN / 32] = {};
         // Classification of pairs hb .. hb+31 (lane l: pair hb + l) for this warp's
         // rows: per 32-column chunk, the pairs some row must correct (tb) and those
         // every row corrects entirely (fb).  Chunks past every row's last valid column
         // (beyond the causal diagonal or the last key, cmax_w) are masked out whole:
         // nothing there needs correcting.  For pairs in [a, u) the windows lie within
         // 127 of the centre, so the thresholds fit in 32 bits.
-        const int cw = SPARSE ? quarter * 32 + static_cast<int>(center) : 0;  // threshold offset of row 0 of the warp
         auto classify = [&](int hb, int& wl, uint32_t (&tb)[BN / 32], uint32_t (&fb)[BN / 32]) {
           const int il = hb + lane;
           const bool valid = il < u;
@@ -512,15 +529,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             fb[qc] = __ballot_sync(0xffffffffu, valid && (addl ? (c_lo >= twl + 31) : (c_lo + 31 < twl)));
           }
         };
-        // the first batch is classified before S arrives, off the softmax -> MMA chain
-        int wl0 = 0;
-        uint32_t tb0[BN / 32] = {}, fb0[BN / 32] = {};
-        if (SPARSE && a < u) classify(a, wl0, tb0, fb0);
-        if (!(ok = warp_wait(&sh->s_full[g], (j - j0) & 1, abort, p.err, 0x303))) break;
+        if constexpr (CORR) {
+          qr = ww.quarter_ranges(center, quarter);
+          z = static_cast<int>(qr & 0xFF);
+          a = static_cast<int>((qr >> 8) & 0xFF);
+          u = static_cast<int>((qr >> 16) & 0xFF);
+          // the next tile's zero point, computed while S is still on its way
+          qr_next = j + 1 < T ? ww.quarter_ranges(center + BN, quarter) : 0u;
+          // no S MMA when every pair is zeroed in every row
+          has_mma = (ww.below(center + kZeroOffset) >> 3) < C::NCH;
+          cnt += static_cast<unsigned long long>(a) * nv;
+          cmax_w = a < u ? __reduce_max_sync(0xffffffffu, cmax) : 0;
+          cw = quarter * 32 + static_cast<int>(center);  // threshold offset of row 0 of the warp
+          // the first batch is classified before S arrives, off the softmax -> MMA chain
+          if (a < u) classify(a, wl0, tb0, fb0);
+        }
+        if (!warp_wait(&sh->s_full[g], (j - j0) & 1, abort, p.err, 0x303)) return false;
         tc_fence_after();
-        uint32_t s_chunks = has_mma ? 0xFu : 0u;  // 32-column chunks of S held in TMEM
-        if (SPARSE) {
-          if (__builtin_expect(a < u, 0)) {
+        if constexpr (CORR) {
+          uint32_t s_chunks = has_mma ? 0xFu : 0u;  // 32-column chunks of S held in TMEM
+          if (a < u) {
             // ---- boundary corrections, in place on S in TMEM, 32 columns at a time.
             const int cen = static_cast<int>(center);
             const uint32_t kbase = smem_u32(sK + s * C::TILE_BYTES);
@@ -616,16 +644,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tmem_st_wait();
           }
-        }
-        if (SPARSE && __builtin_expect(s_chunks != 0xFu, 0)) {
-          // no S MMA on this tile: the chunks no correction wrote hold zero logits
-          uint32_t zw[32];
+          if (s_chunks != 0xFu) {
+            // no S MMA on this tile: the chunks no correction wrote hold zero logits
+            uint32_t zw[32];
 #pragma unroll
-          for (int cc = 0; cc < 32; ++cc) zw[cc] = 0u;
+            for (int cc = 0; cc < 32; ++cc) zw[cc] = 0u;
 #pragma unroll 1
-          for (int qc = 0; qc < BN / 32; ++qc)
-            if (!((s_chunks >> qc) & 1u)) tmem_st32(s_tmem + 32 * qc, zw);
-          tmem_st_wait();
+            for (int qc = 0; qc < BN / 32; ++qc)
+              if (!((s_chunks >> qc) & 1u)) tmem_st32(s_tmem + 32 * qc, zw);
+            tmem_st_wait();
+          }
         }
         // ---- the whole row of S in registers
         float v[BN];
@@ -634,18 +662,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh->k_empty[s]);  // this warp is done with K(j)
-        if (SPARSE && j + 1 < T) {
-          // S_g(j) is done reading Q~_g and this tile's corrections are done with
-          // the stash: zero (and stash) the pairs that die at the next tile.
-          // S_g(j+1) is issued only after this warpgroup's p_full arrival below.
-          const int zn = static_cast<int>(qr_next & 0xFF);
-          if (zn > z) {
-            zero_pairs(sQg, sh->stash[g], r, z, zn);
-            fence_proxy_async_smem();
+        if constexpr (CORR) {
+          if (j + 1 < T) {
+            // S_g(j) is done reading Q~_g and this tile's corrections are done with
+            // the stash: zero (and stash) the pairs that die at the next tile.
+            // S_g(j+1) is issued only after this warpgroup's last P arrival below.
+            const int zn = static_cast<int>(qr_next & 0xFF);
+            if (zn > z) {
+              zero_pairs(sQg, sh->stash[g], r, z, zn);
+              fence_proxy_async_smem();
+            }
+            zst = z;
           }
-          zst = z;
         }
-        qr = qr_next;
 
         // ---- mask, max, exponentials
         if (partial) {
@@ -653,30 +682,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < BN; ++c)
             if (c > cmax) v[c] = -INFINITY;
         }
+        // Row max in eight accumulators: columns 0..7, then 60 steps of two columns.
         float acc[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = fmax3(v[k], v[8 + k], v[16 + k]);
-#pragma unroll
-        for (int c = 24; c < BN - 8; c += 16)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) acc[k] = fmax3(acc[k], v[c + k], v[c + 8 + k]);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = fmaxf(acc[k], v[BN - 8 + k]);
-        const float mx =
-            fmaxf(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], fmax3(acc[5], acc[6], acc[7]))) * scale;
-
-        const float mnew = fmaxf(mrun, mx);
-        // Conditional rescale: keep the stale max until the row max has grown by
-        // more than 2^8; the final 1/l uses the same reference, so this is exact.
-        bool need = false;
-        float corr = 1.f;
-        if (mrun == -INFINITY) {
-          mrun = mnew;
-        } else if (mnew > mrun + 8.f) {
-          need = true;
-          corr = ex2_approx(mrun - mnew);
-        }
-        if (__any_sync(0xffffffffu, need)) {
+        for (int e = 0; e < 8; ++e) acc[e] = v[e];
+        auto max_step = [&](int st) { acc[st & 7] = fmax3(acc[st & 7], v[8 + 2 * st], v[9 + 2 * st]); };
+        auto row_max = [&]() {
+          return fmaxf(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], fmax3(acc[5], acc[6], acc[7]))) * scale;
+        };
+        uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
+        uint32_t pw[BN / 2];
+        const uint64_t sc2 = pack2(scale, scale);
+        uint64_t nm2 = 0ull;  // (-reference, -reference), set once the tile's max is known
+        // P of columns 2k, 2k+1 against the current reference
+        auto exp_pair = [&](int k) {
+          const uint64_t x2 = ffma2(pack2(v[2 * k], v[2 * k + 1]), sc2, nm2);
+          float p0, p1;
+          if (exp_on_fma(k)) {
+            unpack2(exp2_poly2(x2), p0, p1);
+          } else {
+            float x0, x1;
+            unpack2(x2, x0, x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          ls[k & 3] = fadd2(ls[k & 3], pack2(p0, p1));
+          pw[k] = pack_bf16x2(p0, p1);
+        };
+        // Conditional rescale: the reference (mrun) moves only when the row max has
+        // grown by more than 2^8; the final 1/l uses the same reference, so this is
+        // exact.
+        constexpr int KP = BN / 2 / kPPieces;  // column pairs per piece of P
+        // a row's reference moves to mnew: O and l are rescaled by 2^(old - new)
+        // (0 from a row that had no valid column yet, where O and l are 0)
+        auto rescale = [&](float mnew, bool need) {
+          const float corr = need ? ex2_approx(mrun - mnew) : 1.f;
           // O_g holds PV_g up to tile j-1, issued before S_g(j); S_g(j)'s commit
           // covers every earlier MMA, so O_g is complete here.
 #pragma unroll 1
@@ -692,39 +732,62 @@ __global__ void __launch_bounds__(kThreads, 1)
             lsum2 = fmul2(lsum2, pack2(corr, corr));
             mrun = mnew;
           }
-        }
-        const float mref = (mrun == -INFINITY) ? 0.f : mrun;
-        const uint64_t sc2 = pack2(scale, scale), nm2 = pack2(-mref, -mref);
-        uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
-        uint32_t pw[BN / 2];
+        };
 #pragma unroll
-        for (int k = 0; k < BN / 2; ++k) {
-          if (k == BN / 4) {  // first half of P (keys 0..63) is complete: hand it over
-            tmem_st32(s_tmem, pw);
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&sh->p_half[g]);
-          }
-          const uint64_t x2 = ffma2(pack2(v[2 * k], v[2 * k + 1]), sc2, nm2);
-          float p0, p1;
-          if (exp_on_fma(k)) {
-            unpack2(exp2_poly2(x2), p0, p1);
-          } else {
-            float x0, x1;
-            unpack2(x2, x0, x1);
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
-          ls[k & 3] = fadd2(ls[k & 3], pack2(p0, p1));
-          pw[k] = pack_bf16x2(p0, p1);
+        for (int st = 0; st < 60; ++st) max_step(st);
+        const float mnew = fmaxf(mrun, row_max());
+        if (j == j0) {
+          mrun = mnew;  // no reference yet: it is this tile's max
+        } else {
+          // a row that had no valid column yet (mrun = -inf) takes its first reference
+          const bool need = mrun == -INFINITY ? mnew != -INFINITY : mnew > mrun + 8.f;
+          if (__any_sync(0xffffffffu, need)) rescale(mnew, need);
         }
-        tmem_st32(s_tmem + 32, pw + 32);
-        lsum2 = fadd2(lsum2, fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3])));
+        const float mref = mrun == -INFINITY ? 0.f : mrun;
+        nm2 = pack2(-mref, -mref);
+#pragma unroll
+        for (int k = 0; k < KP; ++k) exp_pair(k);
+        // the first piece of P (keys 0..63) goes over while the second is computed
+        tmem_st32(s_tmem, pw);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&sh->p_full[g]);
-      }
+        mbar_arrive(&sh->p_bar[g][0]);
+#pragma unroll
+        for (int k = KP; k < BN / 2; ++k) exp_pair(k);
+        tmem_st32(s_tmem + KP, pw + KP);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&sh->p_bar[g][1]);
+        lsum2 = fadd2(lsum2, fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3])));
+        return true;
+      };
 
+      // Tiles are visited from the diagonal towards key 0.  A run of clean tiles
+      // for this warp ends at the first tile whose distance range [lo, lo + 207)
+      // -- lo = centre + 32 quarter - 127, the smallest distance of the warp's
+      // elements; lo + 207 reaches the next tile's zero point -- holds some window
+      // W_i: there a boundary crosses the warp's elements or pairs die next tile.
+      // The first window not below lo is the next one to enter that range (W is
+      // non-decreasing), so the run length follows from it directly.
+      int j = j0;
+      while (ok && j < T) {
+        int jn = T, a_run = 0;
+        if constexpr (SPARSE) {
+          const long long lo = centre(j + g) + 32 * quarter - (BN - 1);
+          a_run = ww.below(lo);  // pairs dead for every element of the run
+          if (a_run >= C::NP) {
+            jn = j;  // every pair dead: the correcting body handles tiles without S
+          } else {
+            const long long excess = ww.at(a_run) - lo - 206;  // tile j + t holds W when 128 t >= excess
+            jn = excess <= 0 ? j : j + static_cast<int>(min((excess + BN - 1) / BN, static_cast<long long>(T - j)));
+          }
+        }
+        for (; ok && j < jn; ++j) ok = tile(j, std::false_type{}, a_run);
+        if (ok && j < T) {
+          ok = tile(j, std::true_type{}, 0);
+          ++j;
+        }
+      }
       // ---- epilogue: O_g / l -> bf16
       if (ok && warp_wait(&sh->o_done[g], 0, abort, p.err, 0x304)) {
         tc_fence_after();
