@@ -18,22 +18,24 @@ Readings of what the page leaves open:
 - FAC is plain softmax attention, (1/sqrt d) q.k over all d dims, on the selected
   keys and their values.
 
-The selection is an integer decision taken on floating-point scores, so both
-sides take it on the same fp32 numbers: starting from +0, the dims of the
-dominant pairs are taken in ascending order (2i, then 2i+1, pairs ascending)
-and each adds its product with one fused multiply-add in fp32,
-s <- fl(q_j * k_j + s).  Here that rounding is reproduced in fp64: q_j * k_j (a
-bf16 x bf16 product, 16 significant bits) and s (24 bits) sum exactly in fp64
-whenever their exponents are within 28 of each other; otherwise the smaller
-term is below a quarter of an fp32 ulp of the larger, which is itself an fp32
-number, and both roundings return it.  So fp32(fp64(s) + fp64(q_j) * fp64(k_j))
-is exactly the fused result.  FAC itself is fp64.
+The scores here are the exact partial dot products, in fp64 (a bf16 x bf16
+product is exact in fp64, and so is the sum of at most 128 of them whose
+magnitudes stay within 2^29 of each other -- below that the error is far under
+any fp32 rounding).  A GPU computes them in fp32, so its selection is one of
+possibly several correct ones where scores lie within rounding of each other:
+``check_selection`` states which selections are correct (count and order; no
+dropped key scoring above a kept one by more than the two keys' fp32 bounds;
+the lower index first among keys whose dominant dims are identical), and
+``score_bound`` gives the bound: an fp32 sum of n products, each added with one
+rounding, is within n * 2^-24 * sum |q_j k_j| of the exact sum.  FAC is fp64.
 
-Pins (tests/test_fasa_oracle_cpu.py): the all-pairs score equals the full dot
-product within fp32 summation error; a one-pair score equals that pair's
-product sum; a planted monotone score selects the last keys; all-equal scores
-select the first keys; the selection equals a brute-force sort; FAC over every
-token equals the oracle's dense decode; FAC over one token returns its value.
+Pins (tests/test_fasa_oracle_cpu.py): the all-pairs score is the full dot
+product; a one-pair score is that pair's product sum; pairs outside the mask do
+not change a score; a planted monotone score selects the last keys; all-equal
+scores select the first keys; the selection equals a brute-force sort; the
+bound holds for fp32 sums taken in any order; check_selection accepts the
+oracle's selection and rejects planted wrong ones; FAC over every token equals
+the oracle's dense decode; FAC over one token returns its value.
 """
 from __future__ import annotations
 
@@ -68,28 +70,46 @@ def pair_list(mask: int, d: int) -> list[int]:
     return [i for i in range(d // 2) if (mask >> i) & 1]
 
 
+def _masked_dims(mask: int, d: int) -> np.ndarray:
+    return np.array([j for i in pair_list(mask, d) for j in (2 * i, 2 * i + 1)], dtype=np.int64)
+
+
 def tip_scores(q_rot, k_rot, kv_len, mask: int) -> np.ndarray:
-    """TIP scores, float32 [B][Hq][N]; entries at n >= kv_len[b] are -inf.
+    """Exact TIP scores, float64 [B][Hq][N]; entries at n >= kv_len[b] are -inf.
 
     q_rot [B][Hq][d] and k_rot [B][N][Hkv][d] are rotated (interleaved pairs);
     query head h reads kv head h // (Hq / Hkv)."""
-    q = _f32(q_rot)
-    k = _f32(k_rot)
+    q = _f64(q_rot)
+    k = _f64(k_rot)
     B, Hq, d = q.shape
     _, N, Hkv, _ = k.shape
     G = Hq // Hkv
     kl = np.asarray(kv_len, dtype=np.int64).reshape(-1)
-    out = np.full((B, Hq, N), -np.inf, dtype=np.float32)
-    pairs = pair_list(mask, d)
+    out = np.full((B, Hq, N), -np.inf, dtype=np.float64)
+    dims = _masked_dims(mask, d)
     for b in range(B):
         L = int(kl[b])
         for h in range(Hq):
-            kk = k[b, :L, h // G, :]  # [L][d]
-            s = np.zeros(L, dtype=np.float32)
-            for i in pairs:
-                for j in (2 * i, 2 * i + 1):  # one fused multiply-add per dim
-                    s = (s.astype(np.float64) + np.float64(q[b, h, j]) * kk[:, j].astype(np.float64)).astype(np.float32)
-            out[b, h, :L] = s + np.float32(0.0)  # -0 and +0 score alike
+            out[b, h, :L] = k[b, :L, h // G][:, dims] @ q[b, h, dims]
+    return out
+
+
+def score_bound(q_rot, k_rot, kv_len, mask: int) -> np.ndarray:
+    """Per-key bound [B][Hq][N] on |fp32 score - exact score| for an fp32 sum of
+    the 2|mask| products taken one rounding at a time: n * 2^-24 * sum |q_j k_j|
+    (0 past kv_len)."""
+    q = _f64(q_rot)
+    k = _f64(k_rot)
+    B, Hq, d = q.shape
+    _, N, Hkv, _ = k.shape
+    G = Hq // Hkv
+    kl = np.asarray(kv_len, dtype=np.int64).reshape(-1)
+    dims = _masked_dims(mask, d)
+    out = np.zeros((B, Hq, N), dtype=np.float64)
+    for b in range(B):
+        L = int(kl[b])
+        for h in range(Hq):
+            out[b, h, :L] = dims.size * 2.0 ** -24 * (np.abs(k[b, :L, h // G][:, dims]) @ np.abs(q[b, h, dims]))
     return out
 
 
@@ -103,7 +123,7 @@ def select(scores: np.ndarray, kv_len, budget: int) -> np.ndarray:
         L = int(kl[b])
         n = np.arange(L)
         for h in range(Hq):
-            order = np.lexsort((n, -scores[b, h, :L].astype(np.float64)))  # primary: score desc
+            order = np.lexsort((n, -np.asarray(scores[b, h, :L], dtype=np.float64)))  # primary: score desc
             keep = np.sort(order[: min(budget, L)])
             out[b, h, : len(keep)] = keep
     return out
@@ -131,9 +151,58 @@ def focused_attention(q_rot, k_rot, v, sel: np.ndarray) -> np.ndarray:
     return out
 
 
+def check_selection(sel, k_rot, kv_len, budget: int, exact: np.ndarray, bound: np.ndarray, mask: int) -> None:
+    """Raises AssertionError unless `sel` [B][Hq][budget] (int) is a correct
+    selection for the exact scores: per (b, h), the first min(budget, kv_len)
+    entries are distinct key indices in [0, kv_len) in ascending order and the
+    rest are -1; no dropped key's exact score exceeds a kept key's by more than
+    the two keys' bounds (bound[b][h][n]); and where a dropped key's dominant
+    dims equal a kept key's exactly (so any evaluation scores them alike), the
+    kept one has the lower index."""
+    sel = np.asarray(sel)
+    k = _f64(k_rot)
+    B, Hq, _ = sel.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    kl = np.asarray(kv_len, dtype=np.int64).reshape(-1)
+    dims = _masked_dims(mask, k.shape[3])
+    for b in range(B):
+        L = int(kl[b])
+        c = min(budget, L)
+        for h in range(Hq):
+            row = sel[b, h]
+            kept = row[:c].astype(np.int64)
+            assert (row[c:] == -1).all(), (b, h, "padding")
+            assert (kept >= 0).all() and (kept < L).all(), (b, h, "range")
+            assert (np.diff(kept) > 0).all(), (b, h, "ascending and distinct")
+            if c == L:
+                continue
+            is_kept = np.zeros(L, dtype=bool)
+            is_kept[kept] = True
+            e, bd = exact[b, h, :L], bound[b, h, :L]
+            # the kernel keeps k over d only if its fp32 score of k is at least that
+            # of d, so e_d - bd_d <= fp32_d <= fp32_k <= e_k + bd_k for every pair
+            drop = np.nonzero(~is_kept)[0]
+            best_drop = drop[np.argmax(e[drop] - bd[drop])]
+            worst_kept = kept[np.argmin(e[kept] + bd[kept])]
+            assert e[best_drop] - bd[best_drop] <= e[worst_kept] + bd[worst_kept], \
+                (b, h, "dropped key", int(best_drop), "outscores kept key", int(worst_kept))
+            # keys with identical dominant dims score identically in any evaluation:
+            # among them, the kept ones must be the lowest indices
+            tie = drop[np.isin(e[drop], e[kept])]
+            if tie.size:
+                kd = k[b, :L, h // G][:, dims]
+                first_drop = {}
+                for n in tie:
+                    first_drop.setdefault(kd[n].tobytes(), int(n))
+                for n in kept[np.isin(e[kept], e[tie])]:
+                    fd = first_drop.get(kd[n].tobytes())
+                    assert fd is None or fd > n, (b, h, "identical keys: kept", int(n), "after dropped", fd)
+
+
 def fasa_decode(q_rot, k_rot, v, kv_len, mask: int, budget: int):
-    """The whole path: (output fp64 [B][Hq][d], selected int32 [B][Hq][budget],
-    scores float32 [B][Hq][N])."""
+    """The whole path on exact scores: (output fp64 [B][Hq][d], selected int32
+    [B][Hq][budget], exact scores float64 [B][Hq][N])."""
     sc = tip_scores(q_rot, k_rot, kv_len, mask)
     sel = select(sc, kv_len, budget)
     return focused_attention(q_rot, k_rot, v, sel), sel, sc

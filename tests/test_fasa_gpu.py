@@ -1,5 +1,16 @@
-"""FASA-style decode (atf_fasa_decode) against the oracle: the scores and the
-selected key indices bit for bit, the output within the bf16 tolerance."""
+"""FASA-style decode (atf_fasa_decode) against the oracle.
+
+The oracle's scores are exact (fp64); the kernel's are fp32, so each kernel score
+must lie within the oracle's fp32 bound of the exact one, the kernel's selection
+must be a correct one for the exact scores (oracle check_selection: count and
+order, no dropped key ahead of a kept one by more than their bounds, lower index
+first among identical keys), and the output must match the oracle's focused
+attention over the kernel's own selection within the bf16 tolerance.
+
+Separately, as a unit check of the kernel's documented arithmetic (include/atf.h:
+from +0, each dominant dim in ascending order adds its product with one fp32
+fused multiply-add), the kernel's scores are compared bit for bit with that
+evaluation reproduced here in fp64 -- not part of the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -36,13 +47,42 @@ def _run(q, k, v, kv_len, mask, budget):
     return out.cpu(), sel.cpu().numpy(), sc.cpu().numpy()
 
 
-def _check(q, k, v, kv_len, mask, budget):
-    out, sel, sc = _run(q, k, v, kv_len, mask, budget)
-    want, wsel, wsc = ofasa.fasa_decode(q, k, v, kv_len, mask, budget)
+def _fp32_fma_scores(q_rot, k_rot, kv_len, mask):
+    """The kernel's stated score arithmetic: float32 [B][Hq][N], -inf past kv_len.
+    A bf16 x bf16 product (16 significant bits) and the fp32 running sum (24 bits)
+    add exactly in fp64 while their exponents are within 28 of each other, and
+    otherwise both roundings return the larger term, so rounding the fp64 sum to
+    fp32 is the fused multiply-add's result."""
+    q = q_rot.float().numpy()
+    k = k_rot.float().numpy()
+    B, Hq, d = q.shape
+    _, N, Hkv, _ = k.shape
+    G = Hq // Hkv
+    out = np.full((B, Hq, N), -np.inf, dtype=np.float32)
+    dims = [j for i in ofasa.pair_list(mask, d) for j in (2 * i, 2 * i + 1)]
     for b, L in enumerate(kv_len):
-        assert np.array_equal(sc[b, :, :L].view(np.uint32), wsc[b, :, :L].view(np.uint32)), b
-    assert np.array_equal(sel, wsel)
+        for h in range(Hq):
+            kk = k[b, :L, h // G, :]
+            acc = np.zeros(L, dtype=np.float32)
+            for j in dims:
+                acc = (acc.astype(np.float64) + np.float64(q[b, h, j]) * kk[:, j].astype(np.float64)).astype(np.float32)
+            out[b, h, :L] = acc + np.float32(0.0)
+    return out
+
+
+def _check(q, k, v, kv_len, mask, budget, bits=True):
+    out, sel, sc = _run(q, k, v, kv_len, mask, budget)
+    exact = ofasa.tip_scores(q, k, kv_len, mask)
+    bound = ofasa.score_bound(q, k, kv_len, mask)
+    for b, L in enumerate(kv_len):
+        assert np.all(np.abs(sc[b, :, :L].astype(np.float64) - exact[b, :, :L]) <= bound[b, :, :L]), b
+    ofasa.check_selection(sel, k, kv_len, budget, exact, bound, mask)
+    want = ofasa.focused_attention(q, k, v, sel)
     assert np.abs(out.double().numpy() - want).max() <= TOL
+    if bits:  # the kernel's documented fp32 arithmetic, bit for bit
+        fs = _fp32_fma_scores(q, k, kv_len, mask)
+        for b, L in enumerate(kv_len):
+            assert np.array_equal(sc[b, :, :L].view(np.uint32), fs[b, :, :L].view(np.uint32)), b
     return sel
 
 
@@ -107,10 +147,4 @@ def test_fasa_full_size_cache():
     q = synth.token_major(71, 902, 0, 1, 1, 28, 128, torch.bfloat16, threads=4)[:, 0].contiguous()
     k = synth.token_major(71, 902, 1, 1, N, 4, 128, torch.bfloat16, threads=4)
     v = synth.token_major(71, 902, 2, 1, N, 4, 128, torch.bfloat16, threads=4)
-    out, sel, sc = _run(q, k, v, [N], LOW16, budget)
-    wsc = ofasa.tip_scores(q, k, [N], LOW16)
-    assert np.array_equal(sc.view(np.uint32), wsc.view(np.uint32))
-    wsel = ofasa.select(wsc, [N], budget)
-    assert np.array_equal(sel, wsel)
-    want = ofasa.focused_attention(q, k, v, wsel)
-    assert np.abs(out.double().numpy() - want).max() <= TOL
+    _check(q, k, v, [N], LOW16, budget, bits=False)

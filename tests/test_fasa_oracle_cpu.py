@@ -19,11 +19,11 @@ def test_all_pairs_score_is_the_full_dot_product():
     q = _bf16((1, 4, 128), 1)
     k = _bf16((1, 50, 2, 128), 2)
     sc = fasa.tip_scores(q, k, [50], (1 << 64) - 1)
-    qd, kd = q.double().numpy(), k.double().numpy()
+    # the full dot product from torch's own fp64 contraction, heads mapped by GQA
+    full = torch.einsum("bngd,bhd->bhng", k.double(), q.double())  # [b][q head][key][kv head]
     for h in range(4):
-        exact = kd[0, :, h // 2, :] @ qd[0, h]
-        bound = 128 * 2.0 ** -24 * (np.abs(kd[0, :, h // 2, :]) @ np.abs(qd[0, h]))  # one rounding per dim
-        assert np.all(np.abs(sc[0, h] - exact) <= bound)
+        want = full[0, h, :, h // 2].numpy()
+        assert np.allclose(sc[0, h], want, rtol=0, atol=1e-12 * (1 + np.abs(want).max()))
 
 
 def test_one_pair_score_is_that_pairs_product_sum():
@@ -34,8 +34,8 @@ def test_one_pair_score_is_that_pairs_product_sum():
     qd, kd = q.double().numpy(), k.double().numpy()
     for b, L in ((0, 30), (1, 17)):
         for h in range(2):
-            want = (qd[b, h, 2 * i] * kd[b, :L, 0, 2 * i] + qd[b, h, 2 * i + 1] * kd[b, :L, 0, 2 * i + 1])
-            assert np.array_equal(sc[b, h, :L], want.astype(np.float32))  # products exact, one rounding
+            want = qd[b, h, 2 * i] * kd[b, :L, 0, 2 * i] + qd[b, h, 2 * i + 1] * kd[b, :L, 0, 2 * i + 1]
+            assert np.array_equal(sc[b, h, :L], want)  # two bf16 products and one sum, exact in fp64
             assert np.all(np.isneginf(sc[b, h, L:]))
 
 
@@ -103,3 +103,100 @@ def test_focused_attention_over_one_token_returns_its_value():
     vd = v.double().numpy()
     for h, n in enumerate((4, 7, 0)):
         assert np.array_equal(got[0, h], vd[0, n, 0])
+
+
+def _fp32_sum(q, k, dims):
+    """fp32 sequential sums of the products over `dims` in that order (products of
+    bf16 numbers are exact in fp32; each addition rounds once)."""
+    acc = np.zeros(k.shape[0], dtype=np.float32)
+    for j in dims:
+        acc = (acc + (np.float32(q[j]) * k[:, j].astype(np.float32)).astype(np.float32)).astype(np.float32)
+    return acc.astype(np.float64)
+
+
+def test_score_bound_holds_for_fp32_sums_in_any_order():
+    """The bound n 2^-24 sum|q_j k_j| covers an fp32 evaluation in any summation
+    order, on random and on cancellation-heavy inputs (large terms that cancel)."""
+    g = np.random.default_rng(20)
+    mask = (1 << 64) - 1
+    for big in (False, True):
+        qf = g.standard_normal((1, 1, 128)).astype(np.float32)
+        kf = g.standard_normal((1, 400, 1, 128)).astype(np.float32)
+        if big:
+            kf[..., 0::2] *= 1e3
+            kf[..., 1::2] = -kf[..., 0::2] * qf[..., None, None, 0::2][0] / np.where(qf[..., 1::2] == 0, 1, qf[..., 1::2])[0, 0]
+        q = torch.from_numpy(qf).to(torch.bfloat16)
+        k = torch.from_numpy(kf).to(torch.bfloat16)
+        exact = fasa.tip_scores(q, k, [400], mask)[0, 0]
+        bound = fasa.score_bound(q, k, [400], mask)[0, 0]
+        qd, kd = q.float().numpy()[0, 0], k.float().numpy()[0, :, 0]
+        dims = np.arange(128)
+        for order in (dims, dims[::-1], g.permutation(128)):
+            got = _fp32_sum(qd, kd, order)
+            assert np.all(np.abs(got - exact) <= bound), (big, np.abs(got - exact).max(), bound.min())
+
+
+def test_check_selection_accepts_correct_and_rejects_wrong_selections():
+    q = _bf16((1, 2, 64), 21)
+    k = _bf16((1, 500, 1, 64), 22)
+    kv_len, mask, budget = [500], 0xFF00FF, 40
+    exact = fasa.tip_scores(q, k, kv_len, mask)
+    bound = fasa.score_bound(q, k, kv_len, mask)
+    sel = fasa.select(exact, kv_len, budget)
+    fasa.check_selection(sel, k, kv_len, budget, exact, bound, mask)  # the oracle's own selection
+
+    def rejects(bad):
+        try:
+            fasa.check_selection(bad, k, kv_len, budget, exact, bound, mask)
+        except AssertionError:
+            return True
+        return False
+
+    # the lowest kept key swapped for the lowest-scoring dropped key
+    bad = sel.copy()
+    kept = bad[0, 0]
+    drop = np.setdiff1d(np.arange(500), kept)
+    worst = kept[np.argmin(exact[0, 0, kept])]
+    loser = drop[np.argmin(exact[0, 0, drop])]
+    bad[0, 0] = np.sort(np.where(kept == worst, loser, kept))
+    assert rejects(bad)
+    # unsorted, duplicated, out of range, wrong padding
+    bad = sel.copy()
+    bad[0, 1, :2] = bad[0, 1, 1::-1]
+    assert rejects(bad)
+    bad = sel.copy()
+    bad[0, 1, 1] = bad[0, 1, 0]
+    assert rejects(bad)
+    bad = sel.copy()
+    bad[0, 1, -1] = 500
+    assert rejects(bad)
+    short = fasa.select(exact, [30], budget)
+    fasa.check_selection(short, k, [30], budget, fasa.tip_scores(q, k, [30], mask), fasa.score_bound(q, k, [30], mask),
+                         mask)
+    short[0, 0, 35] = 3
+    try:
+        fasa.check_selection(short, k, [30], budget, fasa.tip_scores(q, k, [30], mask),
+                             fasa.score_bound(q, k, [30], mask), mask)
+        raise RuntimeError("padding not checked")
+    except AssertionError:
+        pass
+
+
+def test_check_selection_enforces_the_lower_index_among_identical_keys():
+    q = torch.zeros(1, 1, 64)
+    q[0, 0, 2 * 5] = 1.0
+    k = torch.zeros(1, 10, 1, 64)
+    k[0, :, 0, 2 * 5] = torch.tensor([3.0, 1, 1, 1, 0, 0, 1, 2, 0, 1])
+    q, k = q.to(torch.bfloat16), k.to(torch.bfloat16)
+    mask, budget = 1 << 5, 4  # keys 0 (3), 7 (2), then two of the five keys scoring 1
+    exact = fasa.tip_scores(q, k, [10], mask)
+    bound = fasa.score_bound(q, k, [10], mask)
+    good = np.array([[[0, 1, 2, 7]]], dtype=np.int32)
+    assert np.array_equal(fasa.select(exact, [10], budget), good)
+    fasa.check_selection(good, k, [10], budget, exact, bound, mask)
+    bad = np.array([[[0, 1, 6, 7]]], dtype=np.int32)  # key 6 kept while the identical key 2 is dropped
+    try:
+        fasa.check_selection(bad, k, [10], budget, exact, bound, mask)
+        raise RuntimeError("tie rule not checked")
+    except AssertionError:
+        pass
