@@ -35,6 +35,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -682,11 +683,12 @@ template <int D>
 cudaError_t launch_fasa(const FasaParams& p, long long max_len, cudaStream_t s) {
   const int G = p.hq / p.hkv;
   const size_t hist_smem = static_cast<size_t>(G) * (kHistBins / 2) * sizeof(unsigned int);
-  static unsigned long long configured = 0;  // one bit per device: the attribute is set once
+  // one bit per device: the attribute is set once (racing first calls both set it, harmlessly)
+  static std::atomic<unsigned long long> configured{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 64 || !(configured & (1ull << dev))) {
+  if (dev >= 64 || !(configured.load(std::memory_order_acquire) & (1ull << dev))) {
     const int bytes = kMaxG * (kHistBins / 2) * static_cast<int>(sizeof(unsigned int));
     const void* fns[8] = {reinterpret_cast<const void*>(fasa_score_kernel<D, 1>),
                           reinterpret_cast<const void*>(fasa_score_kernel<D, 2>),
@@ -700,7 +702,7 @@ cudaError_t launch_fasa(const FasaParams& p, long long max_len, cudaStream_t s) 
       e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
       if (e != cudaSuccess) return e;
     }
-    if (dev < 64) configured |= 1ull << dev;
+    if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_acq_rel);
   }
   const unsigned nblk = static_cast<unsigned>((max_len + kScoreKeys - 1) / kScoreKeys);
   const dim3 grid(nblk, p.hkv, p.batch);
