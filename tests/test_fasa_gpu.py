@@ -132,6 +132,31 @@ def test_fasa_lists_longer_than_a_scan_block_stages():
     assert (sel[0, 0] == np.arange(4000)).all() and (sel[0, 1] == np.arange(4000)).all()
 
 
+def test_fasa_unrepresentative_sample_falls_back_to_every_key():
+    """The threshold comes from sampled keys (the first 32 of every 512).  Here
+    only the sampled keys score high, so fewer keys than the budget reach the
+    threshold and the selection is redone over every key's score: the sampled
+    keys plus the best of the rest, and the output from those."""
+    B, N, Hq, Hkv, d = 1, 20000, 3, 1, 64
+    g = np.random.default_rng(13)
+    q = torch.zeros(B, Hq, d)
+    q[:, :, 2 * 5] = 1.0
+    q[:, 1, 2 * 5 + 1] = 0.25
+    q[:, 2, 2 * 5] = -1.0
+    k = torch.from_numpy(0.1 * g.standard_normal((B, N, Hkv, d)).astype(np.float32))
+    sampled = (np.arange(N) % 512) < 32
+    k[0, sampled, 0, 2 * 5] = 4.0
+    v = torch.from_numpy(g.standard_normal((B, N, Hkv, d)).astype(np.float32))
+    q, k, v = q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+    budget = 2048
+    sel = _check(q, k, v, [N], 1 << 5, budget)
+    n_sampled = int(sampled.sum())
+    assert n_sampled < budget
+    for h in (0, 1):  # every sampled key is kept, and budget - n_sampled others
+        assert np.isin(np.nonzero(sampled)[0], sel[0, h]).all()
+    assert not np.isin(np.nonzero(sampled)[0], sel[0, 2]).any()  # head 2 scores them lowest
+
+
 def test_fasa_without_optional_outputs_gives_the_same_result():
     q, k, v = _inputs(2, 4096, 8, 2, 128, seed=67)
     kv_len, budget = [4096, 2500], 300
