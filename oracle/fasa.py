@@ -26,14 +26,27 @@ possibly several correct ones where scores lie within rounding of each other:
 ``check_selection`` states which selections are correct (count and order; no
 dropped key scoring above a kept one by more than the two keys' fp32 bounds;
 the lower index first among keys whose dominant dims are identical), and
-``score_bound`` gives the bound: an fp32 sum of n products, each added with one
-rounding, is within n * 2^-24 * sum |q_j k_j| of the exact sum.  FAC is fp64.
+``score_bound`` gives the bound for one of two ways of summing in fp32:
+- "fma": the n products added one at a time, each with one rounding: within
+  n * 2^-24 * sum |q_j k_j| of the exact sum, in any order;
+- "tensor": the dominant dims grouped by 16-dim cache chunk (pairs 8c .. 8c+7),
+  each chunk's products added to the running fp32 sum in one step.  Assumed of
+  such a step (a hardware adder that aligns its 17 addends to the largest one
+  and keeps at least 24 bits of each): its result is within 18 * 2^-23 of the
+  largest addend's magnitude of the exact step result.  Over C chunks this gives
+  18 * 2^-23 * C * sum |q_j k_j| (times 1 + 2^-16 for the running sum's own
+  error), plus C * 2^-120 for products below fp32's normal range.  This is a
+  stated model, not a documented property: the GPU tests check every kernel
+  score against it.
+FAC is fp64.
 
 Pins (tests/test_fasa_oracle_cpu.py): the all-pairs score is the full dot
 product; a one-pair score is that pair's product sum; pairs outside the mask do
 not change a score; a planted monotone score selects the last keys; all-equal
 scores select the first keys; the selection equals a brute-force sort; the
-bound holds for fp32 sums taken in any order; check_selection accepts the
+"fma" bound holds for fp32 sums taken in any order, and the "tensor" bound for
+a simulated chunk-step adder that truncates every addend below the largest
+one's 24th bit; check_selection accepts the
 oracle's selection and rejects planted wrong ones; FAC over every token equals
 the oracle's dense decode; FAC over one token returns its value.
 """
@@ -94,10 +107,9 @@ def tip_scores(q_rot, k_rot, kv_len, mask: int) -> np.ndarray:
     return out
 
 
-def score_bound(q_rot, k_rot, kv_len, mask: int) -> np.ndarray:
-    """Per-key bound [B][Hq][N] on |fp32 score - exact score| for an fp32 sum of
-    the 2|mask| products taken one rounding at a time: n * 2^-24 * sum |q_j k_j|
-    (0 past kv_len)."""
+def score_bound(q_rot, k_rot, kv_len, mask: int, model: str = "fma") -> np.ndarray:
+    """Per-key bound [B][Hq][N] on |fp32 score - exact score| (0 past kv_len) for
+    the summation `model` ("fma" or "tensor", described above)."""
     q = _f64(q_rot)
     k = _f64(k_rot)
     B, Hq, d = q.shape
@@ -105,11 +117,18 @@ def score_bound(q_rot, k_rot, kv_len, mask: int) -> np.ndarray:
     G = Hq // Hkv
     kl = np.asarray(kv_len, dtype=np.int64).reshape(-1)
     dims = _masked_dims(mask, d)
+    if model == "fma":
+        rel, absolute = dims.size * 2.0 ** -24, 0.0
+    elif model == "tensor":
+        chunks = len({int(i) // 8 for i in pair_list(mask, d)})
+        rel, absolute = 18 * 2.0 ** -23 * chunks * (1 + 2.0 ** -16), chunks * 2.0 ** -120
+    else:
+        raise ValueError(model)
     out = np.zeros((B, Hq, N), dtype=np.float64)
     for b in range(B):
         L = int(kl[b])
         for h in range(Hq):
-            out[b, h, :L] = dims.size * 2.0 ** -24 * (np.abs(k[b, :L, h // G][:, dims]) @ np.abs(q[b, h, dims]))
+            out[b, h, :L] = rel * (np.abs(k[b, :L, h // G][:, dims]) @ np.abs(q[b, h, dims])) + absolute
     return out
 
 

@@ -40,7 +40,9 @@ atf_status cuda_fail(cudaError_t e, const char* what) {
 
 constexpr int kMaxDevices = 64;
 
-unsigned int* device_error_word() {
+}  // namespace
+
+unsigned int* atf::device_error_word() {
   static unsigned int* addr[kMaxDevices] = {};
   static std::mutex mu;
   int dev = 0;
@@ -53,6 +55,8 @@ unsigned int* device_error_word() {
   }
   return addr[dev];
 }
+
+namespace {
 
 // W_i = ceil(alpha * lambda_i), lambda_i = 2 pi / omega_i, omega_i = theta^(-2i/d), fp64.
 void window_table(int d, double theta, double alpha, long long* W, double* omega) {

@@ -82,6 +82,10 @@ cudaError_t launch_decode_merge(const float* parts, int n_parts, long long rows,
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tm_v, const CUtensorMap& tm_k,
                           cudaStream_t s);
 
+// Device address of the library's error word on the current device (bounded
+// waits record their code there), or NULL without a usable device.
+unsigned int* device_error_word();
+
 // Records a printf-style message as this thread's atf_last_error() and returns st.
 atf_status report_error(atf_status st, const char* fmt, ...);
 

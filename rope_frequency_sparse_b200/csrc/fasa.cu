@@ -5,31 +5,35 @@
 // dominant frequency chunks of section "Funktionale Sparsitaet auf
 // Frequenz-Chunk-Ebene" are given here as a set of RoPE pairs.
 //
-// Every TIP score is one fixed fp32 evaluation: from +0, each dim of the
-// dominant pairs (ascending) adds its product with one fused multiply-add,
-// s <- fl(q_j k_j + s), and -0 counts as +0.  The kept keys are the `budget`
-// highest such scores, equal scores by lower index.  Kernels, per call:
-//   1. fasa_sample_kernel: one CTA per (32768 keys, kv head, sequence) scores the
-//      sampled keys -- the first 32 of every 512 -- for all query heads of the kv
-//      head into a 4096-bin histogram per query head (top 12 bits of the score's
-//      order-preserving bit pattern: sign, exponent and three mantissa bits).
+// Every TIP score is one fixed fp32 evaluation on the tensor cores: the 16 dims
+// of each cache chunk that holds a dominant pair (the other pairs' query dims
+// zeroed) are one mma.sync step of bf16 products accumulated into fp32, chunks
+// in ascending order, in one fixed arrangement of dims and heads (score_tiles);
+// -0 counts as +0.  The kept keys are the `budget` highest such scores, equal
+// scores by lower index.  Kernels, per call:
+//   1. fasa_sample_kernel: one CTA per (131072 keys, kv head, sequence) scores the
+//      sampled keys -- the first 32 of every 1024 -- for all query heads of the
+//      kv head into a 4096-bin histogram per query head (top 12 bits of the
+//      score's order-preserving bit pattern: sign, exponent and three mantissa
+//      bits).
 //   2. fasa_threshold_kernel: per query head, the threshold T is the lower edge
 //      of the bin that holds the sample's k-th largest score, k twice the
 //      sample's share of the budget plus 8, so that about twice the budget of
 //      all keys score at or above T.
 //   3. fasa_score_kernel: one CTA per (8192 keys, kv head, sequence); each warp
-//      owns a segment of 1024 consecutive keys, four per lane at a time (two
-//      packed f32x2 fused multiply-adds: each half rounds as the scalar one
-//      does).  It reads only the 8-pair chunks that hold a dominant pair (32
-//      bytes per key and chunk, coalesced) and appends the keys scoring at or
-//      above T, with their scores, to the segment's list in ascending key order.
+//      owns a segment of 1024 consecutive keys, 128 at a time (8 tiles of 16
+//      keys x all query heads of the kv head).  It reads only the 8-pair chunks
+//      that hold a dominant pair (32 bytes per key and chunk, one 8-byte load
+//      per lane and tile row) and appends the keys scoring at or above T, with
+//      their scores, to the segment's list of that head.
 //   4. fasa_select_kernel: one CTA per (query head, sequence) gathers the
-//      segments' lists in order into shared memory and runs a radix select on the
-//      scores' order-preserving bits for the budget-th largest; the keys above it
-//      and the lowest-index ones equal to it are emitted in list order, which is
-//      ascending.  If fewer than `budget` keys reached T (the sample was not
-//      representative), it recomputes every key's score the same way and selects
-//      over all of them; a list longer than shared memory is selected in place.
+//      segments' lists into shared memory, finds the budget-th largest score by a
+//      radix select on the scores' order-preserving bits (and, among keys equal
+//      to it, the lowest indices by a second one on the index), and sorts the
+//      kept indices.  If fewer than `budget` keys reached T (the sample was not
+//      representative), it recomputes every key's score the same way and
+//      selects over all of them; a list longer than shared memory is selected in
+//      place.
 //   5. fasa_attend_kernel: (split of 128 selected keys, query head, sequence);
 //      each warp copies its 32 keys' K rows (chunk-major pieces) and V rows into
 //      shared memory with asynchronous copies, all in flight at once, computes
@@ -51,9 +55,9 @@ namespace atf {
 namespace {
 
 constexpr int kSampleRun = 32;        // sampled keys: the first kSampleRun of every kSamplePeriod
-constexpr int kSamplePeriod = 512;
-constexpr int kSampleCtaKeys = 32768;  // keys of a sequence per sample CTA (64 runs)
-constexpr int kSampleThreads = 512;  // 16 warps, four runs each
+constexpr int kSamplePeriod = 1024;
+constexpr int kSampleCtaKeys = 131072;  // keys of a sequence per sample CTA (128 runs)
+constexpr int kSampleThreads = 512;  // 16 warps, eight runs each
 constexpr int kThresholdThreads = 256;
 constexpr int kHistBits = 12;
 constexpr int kHistBins = 1 << kHistBits;
@@ -62,6 +66,8 @@ constexpr int kScoreThreads = kScoreWarps * 32;
 constexpr int kSegShift = 10;
 constexpr int kSegKeys = 1 << kSegShift;                  // keys per warp segment
 constexpr int kScoreCtaKeys = kScoreWarps * kSegKeys;     // keys per score CTA
+constexpr int kScoreStages = 3;  // bulk-copy stages per score warp
+constexpr size_t kScoreSmem = static_cast<size_t>(kScoreWarps) * kScoreStages * 128 * 32;
 constexpr int kSelectThreads = 1024;
 constexpr int kSelectCap = 16384;  // candidates a select CTA holds in shared memory
 constexpr int kBins = 256;         // radix digit of the select passes
@@ -82,6 +88,7 @@ struct FasaParams {
   unsigned int* hist;       // [B][Hq][kHistBins] sample histograms
   uint32_t* thr;            // [B][Hq] threshold T as an order-preserving key
   int* sel;                 // [B][Hq][budget], ascending, -1 padded
+  unsigned int* err;        // device error word (bounded waits)
   float* partials;          // [B][Hq][n_split][d + 2]
   int batch, hq, hkv, d, budget, n_split;
   long long n_cache, n_seg, seg_cap;  // seg_cap = n_seg * kSegKeys >= n_cache
@@ -111,60 +118,101 @@ __host__ __device__ __forceinline__ long long sample_rank(long long L, int need)
   return (2LL * need * sample_count(L) + L - 1) / L + 8;
 }
 
-// One cache chunk of the TIP score for KP packed key pairs: for each dominant
-// pair j of chunk c (bits), dims 2j and 2j+1 of the chunk add q_dim * k_dim with
-// one fused multiply-add each, both keys of a pair in one f32x2 instruction
-// (each half rounds as the scalar fused multiply-add does).  kv[2e] and kv[2e+1]
-// hold the chunk's 32 bytes of the keys of pair e; sqf[g * qs + 2j] and
-// sqf[g * qs + 2j + 1] hold q of head g at dims 16c + 2j and 16c + 2j + 1 (the
-// query is read from shared memory as 8-byte broadcasts).
-__device__ __forceinline__ uint32_t chunk_word(const uint4 (&kv)[2], int j) {
-  return j == 0 ? kv[0].x : j == 1 ? kv[0].y : j == 2 ? kv[0].z : j == 3 ? kv[0].w
-       : j == 4 ? kv[1].x : j == 5 ? kv[1].y : j == 6 ? kv[1].z : kv[1].w;
-}
-template <int G, int KP>
-__device__ __forceinline__ void score_chunk(const uint4 (&kv)[2 * KP][2], uint32_t bits, const float* sqf, int qs,
-                                            uint64_t (&s2)[KP][G]) {
+// TIP scores on the tensor cores.  One mma.sync m16n8k16 (bf16 in, fp32
+// accumulate) takes a tile of 16 keys x the 16 dims of one cache chunk (A, row =
+// key) against the same 16 dims of the kv head's query heads (B, column = query
+// head g of the group, zero for g >= G and for non-dominant pairs).  The chunks
+// holding a dominant pair are taken in ascending order, each accumulating into
+// the same fp32 fragment.  Within a chunk, lane (g, t) = (lane / 4, lane % 4)
+// supplies words 2t and 2t+1 of its keys' 32-byte chunk rows (dims 4t .. 4t+3)
+// as k-slots (2t, 2t+1) and (2t+8, 2t+9), and the same dims of the query as B --
+// a fixed arrangement, so every kernel that scores a key gets the same bits.
+// Result fragment: c[0], c[1] = key g of the tile, heads 2t and 2t+1; c[2],
+// c[3] = key g+8, heads 2t and 2t+1.
+template <int NC>
+struct QFrag {
+  uint32_t b[NC][2];
+};
+
+// The B fragments of query heads row0 .. row0+G-1 for every chunk.
+template <int D>
+__device__ __forceinline__ QFrag<D / 16> load_qfrag(const __nv_bfloat16* q, long long row0, int G,
+                                                    unsigned long long mask, int lane) {
+  constexpr int NC = D / 16;
+  QFrag<NC> f;
+  const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (!((bits >> j) & 1u)) continue;
-    uint64_t k0[KP], k1[KP];  // dim 2j and dim 2j+1 of the key pairs
-#pragma unroll
-    for (int e = 0; e < KP; ++e) {
-      const uint32_t w0 = chunk_word(kv[2 * e], j), w1 = chunk_word(kv[2 * e + 1], j);
-      k0[e] = pack2(bf16lo_to_f32(w0), bf16lo_to_f32(w1));
-      k1[e] = pack2(bf16hi_to_f32(w0), bf16hi_to_f32(w1));
+  for (int c = 0; c < NC; ++c) {
+    uint32_t lo = 0u, hi = 0u;
+    if (g < G) {
+      const uint32_t* qw = reinterpret_cast<const uint32_t*>(q + (row0 + g) * D + 16 * c + 4 * t);
+      if ((mask >> (8 * c + 2 * t)) & 1ull) lo = __ldg(qw);
+      if ((mask >> (8 * c + 2 * t + 1)) & 1ull) hi = __ldg(qw + 1);
     }
+    f.b[c][0] = lo;
+    f.b[c][1] = hi;
+  }
+  return f;
+}
+
+// Writes the B fragments of load_qfrag to sqf[c][lane] (one warp).
+template <int D>
+__device__ __forceinline__ void store_qfrag(uint2 (*sqf)[32], const __nv_bfloat16* q, long long row0, int G,
+                                            unsigned long long mask, int lane) {
+  const QFrag<D / 16> f = load_qfrag<D>(q, row0, G, mask, lane);
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float2 q2 = *reinterpret_cast<const float2*>(sqf + g * qs + 2 * j);
-      const uint64_t qa = pack2(q2.x, q2.x), qb = pack2(q2.y, q2.y);
+  for (int c = 0; c < D / 16; ++c) sqf[c][lane] = make_uint2(f.b[c][0], f.b[c][1]);
+}
+
+// Scores NT tiles of 16 keys in groups of P consecutive tiles (tile i: keys
+// first + (i / P) * stride + 16 (i % P) .. + 15; keys at or past L read as zero
+// unless `whole` says none is) for the kv head whose chunk-major planes start at
+// kbase, with the B fragments in sqf.  The chunks holding a dominant pair
+// (chunk_mask) are visited in ascending order.
+template <int NT, int P>
+__device__ __forceinline__ long long tile_first(long long first, long long stride, int i) {
+  return first + (i / P) * stride + 16 * (i % P);
+}
+template <int NT, int P>
+__device__ __forceinline__ void score_tiles(float (&acc)[NT][4], const uint2 (*sqf)[32], const __nv_bfloat16* kbase,
+                                            long long n_cache, uint32_t chunk_mask, long long first, long long stride,
+                                            bool whole, long long L, int lane) {
+  const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-      for (int e = 0; e < KP; ++e) {
-        s2[e][g] = ffma2(qa, k0[e], s2[e][g]);
-        s2[e][g] = ffma2(qb, k1[e], s2[e][g]);
+  for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  for (uint32_t cm = chunk_mask; cm; cm &= cm - 1u) {
+    const int c = __ffs(cm) - 1;
+    const uint2 qb = sqf[c][lane];
+    const __nv_bfloat16* row = kbase + (static_cast<long long>(c) * n_cache + first + g) * 16 + 4 * t;
+    uint32_t a[NT][4];
+    if (whole) {
+#pragma unroll
+      for (int i = 0; i < NT; ++i) {
+        const long long off = (tile_first<NT, P>(0, stride, i)) * 16;
+        const uint2 w0 = __ldg(reinterpret_cast<const uint2*>(row + off));
+        const uint2 w1 = __ldg(reinterpret_cast<const uint2*>(row + off + 8 * 16));
+        a[i][0] = w0.x;
+        a[i][1] = w1.x;
+        a[i][2] = w0.y;
+        a[i][3] = w1.y;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < NT; ++i) {
+        const long long off = tile_first<NT, P>(0, stride, i);
+        const long long n0 = first + off + g;
+        uint2 w0 = make_uint2(0u, 0u), w1 = w0;
+        if (n0 < L) w0 = __ldg(reinterpret_cast<const uint2*>(row + off * 16));
+        if (n0 + 8 < L) w1 = __ldg(reinterpret_cast<const uint2*>(row + off * 16 + 8 * 16));
+        a[i][0] = w0.x;
+        a[i][1] = w1.x;
+        a[i][2] = w0.y;
+        a[i][3] = w1.y;
       }
     }
+#pragma unroll
+    for (int i = 0; i < NT; ++i) mma_bf16_16816(acc[i], a[i], qb.x, qb.y);
   }
-}
-
-// Loads the 32 bytes of chunk c of key n (zeros for n >= L).
-__device__ __forceinline__ void load_key_chunk(uint4 (&kv)[2], const uint4* kbase, long long n_cache, int c,
-                                               long long n, long long L) {
-  if (n < L) {
-    const uint4* row = kbase + (static_cast<long long>(c) * n_cache + n) * 2;
-    kv[0] = __ldg(row);
-    kv[1] = __ldg(row + 1);
-  } else {
-    kv[0] = kv[1] = make_uint4(0, 0, 0, 0);
-  }
-}
-
-// Fills sqf[g][j] = q of query head row0 + g at dim j, as floats.
-template <int D, int G>
-__device__ __forceinline__ void load_q(float (&sqf)[G][D], const __nv_bfloat16* q, long long row0, int tid,
-                                       int nthreads) {
-  for (int i = tid; i < G * D; i += nthreads) sqf[i / D][i % D] = __bfloat162float(q[row0 * D + i]);
 }
 
 template <int D, int G>
@@ -172,84 +220,74 @@ __global__ void __launch_bounds__(kSampleThreads) fasa_sample_kernel(FasaParams 
   constexpr int NC = D / 16;
   constexpr int kRuns = kSampleCtaKeys / kSamplePeriod;
   constexpr int kWarps = kSampleThreads / 32;
-  static_assert(kRuns == 4 * kWarps, "each warp scores four runs, two at a time");
+  constexpr int kRunsPerStep = 4;  // two tiles each
+  static_assert(kRuns % (kWarps * kRunsPerStep) == 0 && kSampleRun == 32, "whole steps of four runs per warp");
   const int kvh = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long long L = p.kv_len[b];
   const int need = L < p.budget ? static_cast<int>(L) : p.budget;
   const long long n0 = static_cast<long long>(blockIdx.x) * kSampleCtaKeys;
   if (need == L || n0 >= L) return;  // nothing to select, or no key of this CTA
-  __shared__ __align__(16) float sqf[G][D];
+  __shared__ uint2 s_qf[NC][32];
   __shared__ unsigned int s_lo[G], s_hi[G];  // the range of words any sampled key of this CTA touched
   // per head, kHistBins 16-bit counts packed two to a word (a CTA samples at most
-  // 64 runs of 32 keys)
+  // 128 runs of 32 keys)
   extern __shared__ unsigned int shist[];
   const long long row0 = static_cast<long long>(b) * p.hq + kvh * G;
-  load_q<D, G>(sqf, p.q, row0, tid, kSampleThreads);
   for (int i = tid; i < G * (kHistBins / 2); i += kSampleThreads) shist[i] = 0u;
   if (tid < G) {
     s_lo[tid] = kHistBins / 2;
     s_hi[tid] = 0u;
   }
+  if (warp == 0) store_qfrag<D>(s_qf, p.q, row0, G, p.mask, lane);
   __syncthreads();
-
-  const uint4* kbase = reinterpret_cast<const uint4*>(p.kc) +
-                       (static_cast<long long>(b) * p.hkv + kvh) * NC * p.n_cache * 2;
-  unsigned int lo_w[G], hi_w[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    lo_w[g] = kHistBins / 2;
-    hi_w[g] = 0u;
-  }
-  // warp w scores runs (w, w + kWarps), then (w + 2 kWarps, w + 3 kWarps): one
-  // key of each run per lane, the two as a packed pair
+  const __nv_bfloat16* kbase = p.kc + (static_cast<long long>(b) * p.hkv + kvh) * NC * p.n_cache * 16;
+  const int g = lane >> 2, t = lane & 3;
+  unsigned int lo_w[2] = {kHistBins / 2, kHistBins / 2}, hi_w[2] = {0u, 0u};
+  // warp w, step s: runs (s kWarps + w) kRunsPerStep .. + kRunsPerStep - 1
 #pragma unroll 1
-  for (int h = 0; h < 2; ++h) {
-    const long long na = n0 + static_cast<long long>(warp + 2 * kWarps * h) * kSamplePeriod + lane;
-    const long long nb = na + static_cast<long long>(kWarps) * kSamplePeriod;
-    if (na - lane >= L) break;  // warp-uniform
-    uint64_t s2[1][G];
+  for (int st = 0; st < kRuns / (kWarps * kRunsPerStep); ++st) {
+    const long long first = n0 + static_cast<long long>((st * kWarps + warp) * kRunsPerStep) * kSamplePeriod;
+    if (first >= L) break;  // warp-uniform
+    const bool whole = first + (kRunsPerStep - 1) * kSamplePeriod + kSampleRun <= L;
+    float acc[2 * kRunsPerStep][4];
+    score_tiles<2 * kRunsPerStep, 2>(acc, s_qf, kbase, p.n_cache, p.chunk_mask, first, kSamplePeriod, whole, L, lane);
 #pragma unroll
-    for (int g = 0; g < G; ++g) s2[0][g] = 0ull;
-#pragma unroll 1
-    for (int c = 0; c < NC; ++c) {
-      const uint32_t bits = static_cast<uint32_t>((p.mask >> (8 * c)) & 0xFFu);
-      if (!bits) continue;
-      uint4 kv[2][2];
-      load_key_chunk(kv[0], kbase, p.n_cache, c, na, L);
-      load_key_chunk(kv[1], kbase, p.n_cache, c, nb, L);
-      score_chunk<G, 1>(kv, bits, &sqf[0][16 * c], D, s2);
-    }
+    for (int i = 0; i < 2 * kRunsPerStep; ++i)
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float sc[2];
-      unpack2(s2[0][g], sc[0], sc[1]);
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        if ((e ? nb : na) < L) {
-          const uint32_t bin = order_key(__fadd_rn(sc[e], 0.f)) >> (32 - kHistBits);
-          atomicAdd(&shist[g * (kHistBins / 2) + (bin >> 1)], 1u << (16 * (bin & 1u)));
-          lo_w[g] = min(lo_w[g], bin >> 1);
-          hi_w[g] = max(hi_w[g], bin >> 1);
+      for (int k = 0; k < 4; ++k) {
+        const int h = 2 * t + (k & 1);
+        const long long n = tile_first<2 * kRunsPerStep, 2>(first, kSamplePeriod, i) + g + 8 * (k >> 1);
+        if (h < G && n < L) {
+          const uint32_t bin = order_key(__fadd_rn(acc[i][k], 0.f)) >> (32 - kHistBits);
+          atomicAdd(&shist[h * (kHistBins / 2) + (bin >> 1)], 1u << (16 * (bin & 1u)));
+          lo_w[k & 1] = min(lo_w[k & 1], bin >> 1);
+          hi_w[k & 1] = max(hi_w[k & 1], bin >> 1);
         }
       }
-    }
   }
+  // per head, the touched range over the lanes that hold it (lanes with t = h / 2)
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const unsigned int lo = __reduce_min_sync(0xffffffffu, lo_w[g]), hi = __reduce_max_sync(0xffffffffu, hi_w[g]);
-    if (lane == 0 && lo <= hi) {
-      atomicMin(&s_lo[g], lo);
-      atomicMax(&s_hi[g], hi);
+  for (int e = 0; e < 2; ++e) {
+    unsigned int lo = lo_w[e], hi = hi_w[e];
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    const int h = 2 * t + e;
+    if (g == 0 && h < G && lo <= hi) {
+      atomicMin(&s_lo[h], lo);
+      atomicMax(&s_hi[h], hi);
     }
   }
   __syncthreads();
   // add the touched words' counts to the global histograms
 #pragma unroll 1
-  for (int g = 0; g < G; ++g) {
-    const unsigned int lo = s_lo[g], hi = s_hi[g];
-    unsigned int* hg = p.hist + (row0 + g) * kHistBins;
+  for (int h = 0; h < G; ++h) {
+    const unsigned int lo = s_lo[h], hi = s_hi[h];
+    unsigned int* hg = p.hist + (row0 + h) * kHistBins;
     for (unsigned int i = lo + tid; i <= hi; i += kSampleThreads) {
-      const unsigned int w = shist[g * (kHistBins / 2) + i];
+      const unsigned int w = shist[h * (kHistBins / 2) + i];
       if (w & 0xFFFFu) atomicAdd(&hg[2 * i], w & 0xFFFFu);
       if (w >> 16) atomicAdd(&hg[2 * i + 1], w >> 16);
     }
@@ -307,122 +345,179 @@ __global__ void __launch_bounds__(kThresholdThreads) fasa_threshold_kernel(FasaP
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kScoreThreads, 3) fasa_score_kernel(FasaParams p) {  // 3 CTAs per SM
+__global__ void __launch_bounds__(kScoreThreads, 2) fasa_score_kernel(FasaParams p) {  // 2 CTAs per SM
   constexpr int NC = D / 16;
-  constexpr int KP = 2;                 // packed key pairs per lane
-  constexpr int KU = 2 * KP;            // keys per lane per step
-  constexpr int kStepKeys = 32 * KU;    // keys per warp step
+  constexpr int NT = 8;  // tiles of 16 keys per warp step
+  constexpr int kStepKeys = 16 * NT;
+  constexpr uint32_t kStageBytes = kStepKeys * 32;  // one chunk row of each key of a step
   static_assert(kSegKeys % kStepKeys == 0, "a segment is a whole number of steps");
   const int kvh = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long long L = p.kv_len[b];
   const int need = L < p.budget ? static_cast<int>(L) : p.budget;
   const bool select = need < L;
   if ((!select && !p.scores) || static_cast<long long>(blockIdx.x) * kScoreCtaKeys >= L) return;
-  __shared__ __align__(16) float sqf[G][D];
+  extern __shared__ __align__(128) uint8_t s_ring[];  // per warp: kScoreStages stages of kStageBytes
+  __shared__ uint64_t s_full[kScoreWarps][kScoreStages];
+  __shared__ uint2 s_qf[NC][32];
+  __shared__ float s_tf[8];  // the thresholds as floats
+  __shared__ unsigned int s_cnt[kScoreWarps][8];
+  __shared__ int s_abort;
   const long long row0 = static_cast<long long>(b) * p.hq + kvh * G;
-  load_q<D, G>(sqf, p.q, row0, tid, kScoreThreads);
-  __shared__ float s_tf[G];            // the thresholds as floats
-  __shared__ unsigned int s_cnt[kScoreWarps][G];
-  if (tid < G) s_tf[tid] = select ? key_float(p.thr[row0 + tid]) : 0.f;
-  if (tid < kScoreWarps * G) s_cnt[tid / G][tid % G] = 0u;
+  if (tid < 8) s_tf[tid] = select && tid < G ? key_float(p.thr[row0 + tid]) : 0.f;
+  if (tid < kScoreWarps * 8) s_cnt[tid / 8][tid % 8] = 0u;
+  if (tid < kScoreWarps * kScoreStages) mbar_init(&s_full[tid / kScoreStages][tid % kScoreStages], 1);
+  if (tid == 0) s_abort = 0;
+  if (warp == 0) store_qfrag<D>(s_qf, p.q, row0, G, p.mask, lane);
+  fence_mbar_init();
   __syncthreads();
   const long long wseg = static_cast<long long>(blockIdx.x) * kScoreWarps + warp;
   const long long base = wseg * kSegKeys;
   if (base >= L) return;
   const int n_steps = static_cast<int>(min(static_cast<long long>(kSegKeys / kStepKeys),
                                            (L - base + kStepKeys - 1) / kStepKeys));
-  const uint4* kbase = reinterpret_cast<const uint4*>(p.kc) +
-                       (static_cast<long long>(b) * p.hkv + kvh) * NC * p.n_cache * 2;
   const uint32_t cm = p.chunk_mask;
-  const int c_first = __ffs(cm) - 1;
-  auto next_chunk = [cm](int c) { return __ffs(cm & ~((2u << c) - 1u)) - 1; };
+  const int n_chunks = __popc(cm);
+  const int n_stages = n_steps * n_chunks;  // (step, chunk) pairs, chunk fastest
+  const __nv_bfloat16* kbase = p.kc + (static_cast<long long>(b) * p.hkv + kvh) * NC * p.n_cache * 16;
+  uint8_t* ring = s_ring + static_cast<size_t>(warp) * kScoreStages * kStageBytes;
+  uint64_t* full = s_full[warp];
+  // the c-th set bit of the chunk mask
+  auto nth_chunk = [cm](int k) {
+    uint32_t m = cm;
+    for (int j = 0; j < k; ++j) m &= m - 1u;
+    return __ffs(m) - 1;
+  };
+  auto issue = [&](int q) {  // lane 0: the bulk copy of stage q into slot q % kScoreStages
+    const int it = q / n_chunks, c = nth_chunk(q - it * n_chunks);
+    const long long s0 = base + static_cast<long long>(kStepKeys) * it;
+    const uint32_t bytes = static_cast<uint32_t>(min(static_cast<long long>(kStepKeys), L - s0)) * 32u;
+    uint64_t* bar = &full[q % kScoreStages];
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load(ring + (q % kScoreStages) * kStageBytes, kbase + (static_cast<long long>(c) * p.n_cache + s0) * 16,
+              bytes, bar);
+  };
+  int issued = 0;
+  if (lane == 0)
+    for (; issued < min(kScoreStages, n_stages); ++issued) issue(issued);
+  issued = __shfl_sync(0xffffffffu, issued, 0);
 
-  // KU keys per lane per step: key u is base + kStepKeys * it + 32 u + lane;
-  // keys (2e, 2e+1) are scored as packed pair e
-  auto load = [&](uint4 (&buf)[KU][2], int it, int c) {
-    const long long n0 = base + kStepKeys * it + lane;
+  const int g = lane >> 2, t = lane & 3;
+  const bool hv0 = 2 * t < G, hv1 = 2 * t + 1 < G;
+  const float t0 = s_tf[2 * t], t1 = s_tf[2 * t + 1];
+  unsigned int* err = p.err;
+  int q = 0;
+  bool ok = true;
+  for (int it = 0; it < n_steps && ok; ++it) {
+    const long long s0 = base + static_cast<long long>(kStepKeys) * it;
+    const bool whole = s0 + kStepKeys <= L;
+    float acc[NT][4];
 #pragma unroll
-    for (int u = 0; u < KU; ++u) load_key_chunk(buf[u], kbase, p.n_cache, c, n0 + 32 * u, L);
-  };
-  uint64_t s2[KP][G];
-#pragma unroll
-  for (int e = 0; e < KP; ++e)
-#pragma unroll
-    for (int g = 0; g < G; ++g) s2[e][g] = 0ull;  // (+0, +0)
-  auto compute = [&](const uint4 (&buf)[KU][2], int c) {
-    score_chunk<G, KP>(buf, static_cast<uint32_t>((p.mask >> (8 * c)) & 0xFFu), &sqf[0][16 * c], D, s2);
-  };
-  const unsigned int lt = (1u << lane) - 1u;
-  auto finish_step = [&](int it) {
-    float sc[G][KU];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int e = 0; e < KP; ++e) {
-        unpack2(s2[e][g], sc[g][2 * e], sc[g][2 * e + 1]);
-        s2[e][g] = 0ull;
+    for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    for (int ci = 0; ci < n_chunks; ++ci, ++q) {
+      if (!warp_wait(&full[q % kScoreStages], (q / kScoreStages) & 1, &s_abort, err, 0x501)) {
+        ok = false;
+        break;
       }
-    const long long n0 = base + kStepKeys * it + lane;
-    bool vu[KU];
+      const uint2 qb = s_qf[nth_chunk(ci)][lane];
+      const uint8_t* st = ring + (q % kScoreStages) * kStageBytes + 32 * g + 8 * t;
+      uint32_t a[NT][4];
 #pragma unroll
-    for (int u = 0; u < KU; ++u) vu[u] = n0 + 32 * u < L;
+      for (int i = 0; i < NT; ++i) {
+        uint2 w0 = *reinterpret_cast<const uint2*>(st + 512 * i);
+        uint2 w1 = *reinterpret_cast<const uint2*>(st + 512 * i + 256);
+        if (!whole) {  // the copy stopped at key L - 1
+          if (s0 + 16 * i + g >= L) w0 = make_uint2(0u, 0u);
+          if (s0 + 16 * i + g + 8 >= L) w1 = make_uint2(0u, 0u);
+        }
+        a[i][0] = w0.x;
+        a[i][1] = w1.x;
+        a[i][2] = w0.y;
+        a[i][3] = w1.y;
+      }
+      __syncwarp();  // every lane has read the slot: it may be refilled
+      if (lane == 0 && issued < n_stages) issue(issued);
+      ++issued;
+#pragma unroll
+      for (int i = 0; i < NT; ++i) mma_bf16_16816(acc[i], a[i], qb.x, qb.y);
+    }
+    if (!ok) break;
+    // acc[i][k]: key s0 + 16 i + g + 8 (k >> 1), head 2t + (k & 1)
     if (p.scores) {
 #pragma unroll
-      for (int g = 0; g < G; ++g)
+      for (int i = 0; i < NT; ++i)
 #pragma unroll
-        for (int u = 0; u < KU; ++u)
-          if (vu[u]) p.scores[(row0 + g) * p.n_cache + n0 + 32 * u] = __fadd_rn(sc[g][u], 0.f);
-    }
-    if (!select) return;
-    // !(s < T) holds for s >= T; T is never -0, and a -0 score counts as +0
-    bool any = false;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float t = s_tf[g];
-#pragma unroll
-      for (int u = 0; u < KU; ++u) any |= vu[u] && !(sc[g][u] < t);
-    }
-    if (!__any_sync(0xffffffffu, any)) return;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float t = s_tf[g];
-      unsigned int cnt = s_cnt[warp][g];
-      const long long seg = (row0 + g) * p.seg_cap + base;
-#pragma unroll
-      for (int u = 0; u < KU; ++u) {  // ascending key order within the segment
-        const bool c = vu[u] && !(sc[g][u] < t);
-        const unsigned int bal = __ballot_sync(0xffffffffu, c);
-        if (c) {
-          const unsigned int pos = cnt + static_cast<unsigned int>(__popc(bal & lt));
-          p.cand[seg + pos] = static_cast<uint32_t>(n0 + 32 * u);
-          p.cand_score[seg + pos] = __fadd_rn(sc[g][u], 0.f);
+        for (int k = 0; k < 4; ++k) {
+          const int h = 2 * t + (k & 1);
+          const long long n = s0 + 16 * i + g + 8 * (k >> 1);
+          if (h < G && n < L) p.scores[(row0 + h) * p.n_cache + n] = __fadd_rn(acc[i][k], 0.f);
         }
-        cnt += static_cast<unsigned int>(__popc(bal));
-      }
-      __syncwarp();
-      if (lane == 0) s_cnt[warp][g] = cnt;
-      __syncwarp();
     }
-  };
-
-  // four keys per lane per step, one chunk at a time; three CTAs per SM keep
-  // enough warps in flight to cover the loads (a second register stage for the
-  // next chunk's loads costs more in occupancy than it hides)
-  uint4 buf[KU][2];
-  for (int it = 0; it < n_steps; ++it) {
-    for (int c = c_first; c >= 0; c = next_chunk(c)) {
-      load(buf, it, c);
-      compute(buf, c);
-    }
-    finish_step(it);
-  }
-  if (select && lane < G) {
-    unsigned int v = 0;
+    if (!select) continue;
+    // candidate bits: bit 4i + k for acc[i][k] at or above its head's threshold
+    // (!(s < T) holds for s >= T; T is never -0, and a -0 score counts as +0)
+    uint32_t m = 0u;
+    if (whole) {
 #pragma unroll
-    for (int g = 0; g < G; ++g)
-      if (lane == g) v = s_cnt[warp][g];
-    p.seg_cnt[(row0 + lane) * p.n_seg + wseg] = v;
+      for (int i = 0; i < NT; ++i)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          m |= static_cast<uint32_t>(!(acc[i][k] < ((k & 1) ? t1 : t0))) << (4 * i + k);
+    } else {
+#pragma unroll
+      for (int i = 0; i < NT; ++i)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          m |= static_cast<uint32_t>(!(acc[i][k] < ((k & 1) ? t1 : t0)) && s0 + 16 * i + g + 8 * (k >> 1) < L)
+               << (4 * i + k);
+    }
+    m &= (hv0 ? 0x55555555u : 0u) | (hv1 ? 0xAAAAAAAAu : 0u);
+    if (!__any_sync(0xffffffffu, m != 0u)) continue;
+    // slots: the lanes sharing this lane's two heads (lanes t, t + 4, .., t + 28,
+    // in key order within each tile row) take consecutive runs after the
+    // segment's count; order within a segment is arbitrary (the selection sorts
+    // what it keeps)
+    const int c0 = __popc(m & 0x55555555u), c1 = __popc(m & 0xAAAAAAAAu);
+    int p0 = c0, p1 = c1;
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      const int y0 = __shfl_up_sync(0xffffffffu, p0, off), y1 = __shfl_up_sync(0xffffffffu, p1, off);
+      if (lane >= off) {
+        p0 += y0;
+        p1 += y1;
+      }
+    }
+    const int tot0 = __shfl_sync(0xffffffffu, p0, 28 + t), tot1 = __shfl_sync(0xffffffffu, p1, 28 + t);
+    unsigned int pos0 = s_cnt[warp][2 * t] + static_cast<unsigned int>(p0 - c0);
+    unsigned int pos1 = s_cnt[warp][2 * t + 1] + static_cast<unsigned int>(p1 - c1);
+    __syncwarp();
+    if (g == 0) {
+      s_cnt[warp][2 * t] += static_cast<unsigned int>(tot0);
+      s_cnt[warp][2 * t + 1] += static_cast<unsigned int>(tot1);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+      for (uint32_t mi = (m >> (4 * i)) & 15u; mi; mi &= mi - 1u) {
+        const int k = __ffs(mi) - 1;
+        const float v = k == 0 ? acc[i][0] : k == 1 ? acc[i][1] : k == 2 ? acc[i][2] : acc[i][3];
+        const unsigned int pos = (k & 1) ? pos1++ : pos0++;
+        const long long slot = (row0 + 2 * t + (k & 1)) * p.seg_cap + base + pos;
+        p.cand[slot] = static_cast<uint32_t>(s0 + 16 * i + g + 8 * (k >> 1));
+        p.cand_score[slot] = __fadd_rn(v, 0.f);
+      }
+    }
   }
+  if (!ok) {  // a copy did not land in time: wait (bounded) for this warp's copies still in flight
+    if (lane == 0)
+      for (int r = q; r < min(issued, n_stages); ++r) {
+        const long long w0 = clock64();
+        while (!mbar_try_wait(&full[r % kScoreStages], (r / kScoreStages) & 1) && clock64() - w0 < kWaitLimitCycles) {
+        }
+      }
+    return;
+  }
+  __syncwarp();
+  if (select && lane < G) p.seg_cnt[(row0 + lane) * p.n_seg + wseg] = s_cnt[warp][lane];
 }
 
 // Exclusive prefix sum of v over the kSelectThreads threads; *total gets the sum.
@@ -454,8 +549,8 @@ __device__ __forceinline__ int block_scan(int v, int* s_warp, int* total) {
   return r;
 }
 
-// The candidates of one (query head, sequence) in ascending key order, held in
-// shared memory: order keys and key indices.
+// The candidates of one (query head, sequence), held in shared memory: order
+// keys and key indices.
 struct SmemList {
   const uint32_t* key;
   const uint32_t* idx;
@@ -485,21 +580,22 @@ struct SegmentList {
 
 struct SelectScratch {
   unsigned int* hist;  // kBins
-  int* warp;           // 32
   int* total;
   int* digit;
   int* gt;
+  int* out;            // kMaxFasaBudget
 };
 
-// Writes to out[0 .. need) the indices of the `need` largest entries of `list`
-// (by order key, equal keys by position, the list being in ascending key
-// order), in list order, and -1 to out[need .. budget).  The list holds at
-// least `need` entries.
-template <class List>
-__device__ void select_emit(const List& list, int need, int budget, int* out, const SelectScratch& sc) {
+// Radix select over the 32-bit values val(i) of the entries i of `list` with
+// in(i): returns the value v such that `rank` entries (1 <= rank <= count) lie
+// at or above it in the order of `largest` (descending if true), and writes to
+// *before the number strictly beyond it.  Every thread of the block calls it.
+template <class List, class Val, class In>
+__device__ uint32_t radix_select(const List& list, Val val, In in, int rank, bool largest, int* before,
+                                 const SelectScratch& sc) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t prefix = 0u, pmask = 0u;
-  int left = need;
+  int left = rank, beyond = 0;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     for (int i = tid; i < kBins; i += kSelectThreads) sc.hist[i] = 0u;
@@ -510,28 +606,31 @@ __device__ void select_emit(const List& list, int need, int budget, int* out, co
     __syncthreads();
     for (long long i = tid; i < list.n; i += kSelectThreads) {
       uint32_t k, x;
-      if (list.get(i, k, x) && (k & pmask) == prefix) atomicAdd(&sc.hist[(k >> shift) & (kBins - 1)], 1u);
+      if (list.get(i, k, x) && in(k, x)) {
+        const uint32_t v = val(k, x);
+        if ((v & pmask) == prefix) atomicAdd(&sc.hist[(v >> shift) & (kBins - 1)], 1u);
+      }
     }
     __syncthreads();
     if (warp == 0) {
-      // the digit d: the largest with #(digits >= d) >= left; lane l holds the
-      // digits 8l .. 8l+7, suffix sums across the lanes
+      // the digit d: the first, in the selection order, whose cumulative count
+      // reaches `left`; lane l holds 8 consecutive digits in that order
       int c8 = 0;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) c8 += static_cast<int>(sc.hist[8 * lane + u]);
-      int suf = c8;  // digits >= 8 lane
+      for (int u = 0; u < 8; ++u) c8 += static_cast<int>(sc.hist[largest ? 255 - (8 * lane + u) : 8 * lane + u]);
+      int incl = c8;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_down_sync(0xffffffffu, suf, off);
-        if (lane + off < 32) suf += y;
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
       }
-      const int above = suf - c8;  // digits >= 8 lane + 8
-      if (above < left && left <= suf) {
-        int run = above;
-        for (int u = 8 * lane + 7; u >= 8 * lane; --u) {
-          const int cu = static_cast<int>(sc.hist[u]);
+      if (incl - c8 < left && left <= incl) {
+        int run = incl - c8;
+        for (int u = 0; u < 8; ++u) {
+          const int d = largest ? 255 - (8 * lane + u) : 8 * lane + u;
+          const int cu = static_cast<int>(sc.hist[d]);
           if (run + cu >= left) {
-            *sc.digit = u;
+            *sc.digit = d;
             *sc.gt = run;
             break;
           }
@@ -541,45 +640,79 @@ __device__ void select_emit(const List& list, int need, int budget, int* out, co
     }
     __syncthreads();
     left -= *sc.gt;
+    beyond += *sc.gt;
     prefix |= static_cast<uint32_t>(*sc.digit) << shift;
     pmask |= static_cast<uint32_t>(kBins - 1) << shift;
     __syncthreads();  // digit and gt are rewritten by the next pass
   }
-  // prefix is the need-th largest key; all keys above it are kept, and the first
-  // `left` equal to it in list order.  Thread t emits the contiguous block
-  // [t * per, (t + 1) * per) of the list.
-  const long long per = (list.n + kSelectThreads - 1) / kSelectThreads;
-  const long long lo = tid * per, hi = min(list.n, lo + per);
-  int eq = 0;
-  for (long long i = lo; i < hi; ++i) {
-    uint32_t k, x;
-    if (list.get(i, k, x) && k == prefix) ++eq;
-  }
-  const int eq_before = block_scan(eq, sc.warp, sc.total);
-  int keep = 0, e = eq_before;
-  for (long long i = lo; i < hi; ++i) {
-    uint32_t k, x;
-    if (!list.get(i, k, x)) continue;
-    if (k > prefix) {
-      ++keep;
-    } else if (k == prefix) {
-      keep += e < left;
-      ++e;
-    }
-  }
-  int pos = block_scan(keep, sc.warp, sc.total);
-  e = eq_before;
-  for (long long i = lo; i < hi; ++i) {
-    uint32_t k, x;
-    if (!list.get(i, k, x)) continue;
-    if (k > prefix || (k == prefix && e++ < left)) {
-      if (pos < need) out[pos] = static_cast<int>(x);
-      ++pos;
-    }
-  }
-  for (int i = need + tid; i < budget; i += kSelectThreads) out[i] = -1;
+  *before = beyond;
+  return prefix;
 }
 
+// Writes to out[0 .. need) the indices of the `need` largest entries of `list`
+// by order key (equal keys: lower index first), ascending, and -1 to out[need ..
+// budget).  The list holds at least `need` entries.
+template <class List>
+__device__ void select_emit(const List& list, int need, int budget, int* out, const SelectScratch& sc) {
+  const int tid = threadIdx.x;
+  auto by_key = [](uint32_t k, uint32_t) { return k; };
+  auto all = [](uint32_t, uint32_t) { return true; };
+  int above = 0;
+  const uint32_t V = radix_select(list, by_key, all, need, true, &above, sc);
+  const int left = need - above;  // entries equal to V to keep: the lowest indices
+  // count the entries equal to V; if there are more than `left`, the left-th
+  // smallest index among them decides
+  if (tid == 0) *sc.total = 0;
+  __syncthreads();
+  int eq = 0;
+  for (long long i = tid; i < list.n; i += kSelectThreads) {
+    uint32_t k, x;
+    eq += list.get(i, k, x) && k == V;
+  }
+  if (eq) atomicAdd(sc.total, eq);
+  __syncthreads();
+  uint32_t I = 0xFFFFFFFFu;
+  if (*sc.total > left) {
+    auto by_idx = [](uint32_t, uint32_t x) { return x; };
+    auto equal = [V](uint32_t k, uint32_t) { return k == V; };
+    int below = 0;
+    I = radix_select(list, by_idx, equal, left, false, &below, sc);
+  }
+  __syncthreads();
+  if (tid == 0) *sc.total = 0;
+  __syncthreads();
+  for (long long i = tid; i < list.n; i += kSelectThreads) {
+    uint32_t k, x;
+    if (list.get(i, k, x) && (k > V || (k == V && x <= I))) {
+      const int slot = atomicAdd(sc.total, 1);
+      if (slot < need) sc.out[slot] = static_cast<int>(x);
+    }
+  }
+  __syncthreads();
+  // bitonic sort of the kept indices (padded to a power of two)
+  int P = 1;
+  while (P < need) P <<= 1;
+  for (int i = need + tid; i < P; i += kSelectThreads) sc.out[i] = 0x7fffffff;
+  __syncthreads();
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < P; i += kSelectThreads) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const int a = sc.out[i], c = sc.out[ixj];
+          if ((a > c) == ((i & k) == 0)) {
+            sc.out[i] = c;
+            sc.out[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = tid; i < budget; i += kSelectThreads) out[i] = i < need ? sc.out[i] : -1;
+}
+
+template <int D>
 __global__ void __launch_bounds__(kSelectThreads) fasa_select_kernel(FasaParams p) {
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const long long row = static_cast<long long>(b) * p.hq + h;
@@ -594,8 +727,8 @@ __global__ void __launch_bounds__(kSelectThreads) fasa_select_kernel(FasaParams 
   __shared__ unsigned int s_hist[kBins];
   __shared__ int s_warp[32];
   __shared__ int s_total, s_digit, s_gt;
-  __shared__ float s_q[128];
-  const SelectScratch scr{s_hist, s_warp, &s_total, &s_digit, &s_gt};
+  __shared__ int s_out[kMaxFasaBudget];
+  const SelectScratch scr{s_hist, &s_total, &s_digit, &s_gt, s_out};
   const uint32_t T = p.thr[row];
   const long long nseg = (L + kSegKeys - 1) / kSegKeys;
   const unsigned int* cnt = p.seg_cnt + row * p.n_seg;
@@ -642,30 +775,31 @@ __global__ void __launch_bounds__(kSelectThreads) fasa_select_kernel(FasaParams 
       return;
     }
   }
-  // fewer than `need` keys reached T: every key's score, in the same arithmetic,
-  // into the (now unused) candidate arrays, slot n = key n, then select over all
-  const int D = p.d, NC = D / 16;
-  for (int i = tid; i < D; i += kSelectThreads) s_q[i] = __bfloat162float(p.q[row * D + i]);
-  __syncthreads();
-  const uint4* kbase = reinterpret_cast<const uint4*>(p.kc) +
-                       (static_cast<long long>(b) * p.hkv + h / (p.hq / p.hkv)) * NC * p.n_cache * 2;
-  for (long long n = tid; n < L; n += kSelectThreads) {
-    float s = 0.f;
-    for (int c = 0; c < NC; ++c) {
-      const uint32_t bits = static_cast<uint32_t>((p.mask >> (8 * c)) & 0xFFu);
-      if (!bits) continue;
-      const uint4* r = kbase + (static_cast<long long>(c) * p.n_cache + n) * 2;
-      const uint4 lo = __ldg(r), hi = __ldg(r + 1);
-      const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  // fewer than `need` keys reached T: every key's score, in the same arithmetic
+  // and arrangement as the scoring kernel, into the (now unused) candidate
+  // arrays, slot n = key n, then select over all
+  {
+    constexpr int NC = D / 16;
+    __shared__ uint2 s_qf[NC][32];
+    const int G = p.hq / p.hkv, kvh = h / G, hl = h - kvh * G;
+    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+    if (warp == 0) store_qfrag<D>(s_qf, p.q, static_cast<long long>(b) * p.hq + kvh * G, G, p.mask, lane);
+    __syncthreads();
+    const __nv_bfloat16* kbase = p.kc + (static_cast<long long>(b) * p.hkv + kvh) * NC * p.n_cache * 16;
+    for (long long tile = warp; tile * 16 < L; tile += kSelectThreads / 32) {
+      float acc[1][4];
+      score_tiles<1, 1>(acc, s_qf, kbase, p.n_cache, p.chunk_mask, tile * 16, 0, tile * 16 + 16 <= L, L, lane);
+      if (t == hl / 2) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (!((bits >> j) & 1u)) continue;
-        s = __fmaf_rn(s_q[16 * c + 2 * j], bf16lo_to_f32(w[j]), s);
-        s = __fmaf_rn(s_q[16 * c + 2 * j + 1], bf16hi_to_f32(w[j]), s);
+        for (int r = 0; r < 2; ++r) {
+          const long long n = tile * 16 + g + 8 * r;
+          if (n < L) {
+            cscore[n] = __fadd_rn(acc[0][2 * r + (hl & 1)], 0.f);
+            cand[n] = static_cast<uint32_t>(n);
+          }
+        }
       }
     }
-    cscore[n] = __fadd_rn(s, 0.f);
-    cand[n] = static_cast<uint32_t>(n);
   }
   __syncthreads();
   select_emit(SegmentList{cand, cscore, cnt, L, true}, need, p.budget, out, scr);
@@ -881,7 +1015,7 @@ void launch_select_path(const FasaParams& p, long long max_len, cudaStream_t s) 
   fasa_threshold_kernel<<<dim3(p.hq, p.batch), kThresholdThreads, 0, s>>>(p);
   fasa_score_kernel<D, G><<<dim3(static_cast<unsigned>((max_len + kScoreCtaKeys - 1) / kScoreCtaKeys), p.hkv,
                                  p.batch),
-                            kScoreThreads, 0, s>>>(p);
+                            kScoreThreads, kScoreSmem, s>>>(p);
 }
 
 template <int D>
@@ -908,7 +1042,19 @@ cudaError_t launch_fasa(const FasaParams& p, long long max_len, cudaStream_t s) 
       e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
       if (e != cudaSuccess) return e;
     }
-    e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fasa_select_kernel),
+    const void* score_fns[8] = {reinterpret_cast<const void*>(fasa_score_kernel<D, 1>),
+                                reinterpret_cast<const void*>(fasa_score_kernel<D, 2>),
+                                reinterpret_cast<const void*>(fasa_score_kernel<D, 3>),
+                                reinterpret_cast<const void*>(fasa_score_kernel<D, 4>),
+                                reinterpret_cast<const void*>(fasa_score_kernel<D, 5>),
+                                reinterpret_cast<const void*>(fasa_score_kernel<D, 6>),
+                                reinterpret_cast<const void*>(fasa_score_kernel<D, 7>),
+                                reinterpret_cast<const void*>(fasa_score_kernel<D, 8>)};
+    for (const void* f : score_fns) {
+      e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kScoreSmem));
+      if (e != cudaSuccess) return e;
+    }
+    e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fasa_select_kernel<D>),
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSelectSmem));
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fasa_attend_kernel<D>),
@@ -926,7 +1072,7 @@ cudaError_t launch_fasa(const FasaParams& p, long long max_len, cudaStream_t s) 
     case 7: launch_select_path<D, 7>(p, max_len, s); break;
     default: launch_select_path<D, 8>(p, max_len, s); break;
   }
-  fasa_select_kernel<<<dim3(p.hq, p.batch), kSelectThreads, kSelectSmem, s>>>(p);
+  fasa_select_kernel<D><<<dim3(p.hq, p.batch), kSelectThreads, kSelectSmem, s>>>(p);
   fasa_attend_kernel<D><<<dim3(p.n_split, p.hq, p.batch), kAttendWarps * 32, kAttendSmem, s>>>(p);
   fasa_combine_kernel<D><<<dim3(p.hq, p.batch), D, 0, s>>>(p);
   return cudaGetLastError();
@@ -989,6 +1135,8 @@ extern "C" atf_status atf_fasa_decode(const void* q_rot, const void* k_chunked, 
   p.hist = reinterpret_cast<unsigned int*>(ws + Lw.hist);
   p.thr = reinterpret_cast<uint32_t*>(ws + Lw.thr);
   p.sel = selected ? selected : reinterpret_cast<int*>(ws + Lw.sel);
+  p.err = device_error_word();
+  if (!p.err) return report_error(ATF_ERR_CUDA, "fasa: no CUDA device / device error word unavailable");
   p.partials = reinterpret_cast<float*>(ws + Lw.partials);
   p.batch = batch;
   p.hq = heads;

@@ -136,6 +136,58 @@ def test_score_bound_holds_for_fp32_sums_in_any_order():
             assert np.all(np.abs(got - exact) <= bound), (big, np.abs(got - exact).max(), bound.min())
 
 
+def _chunk_step_sum(qd, kd, chunks):
+    """A model of a 16-dim chunk step: the running sum and the chunk's products
+    aligned to the largest of them, each truncated (toward zero) below that one's
+    24th significant bit, added exactly, the result truncated to fp32."""
+    from fractions import Fraction
+
+    out = np.empty(kd.shape[0], dtype=np.float64)
+    for n in range(kd.shape[0]):
+        run = 0.0
+        for c in chunks:
+            terms = [run] + [float(qd[j]) * float(kd[n, j]) for j in range(16 * c, 16 * c + 16)]
+            big = max(abs(x) for x in terms)
+            if big == 0.0:
+                continue
+            unit = Fraction(2) ** (math.frexp(big)[1] - 24)  # the largest term's 24th significant bit
+            tot = sum(Fraction(math.trunc(Fraction(x) / unit)) * unit for x in terms)
+            run = float(np.float32(float(tot)))  # exact result to fp32; then toward zero
+            if abs(run) > abs(float(tot)):
+                run = float(np.nextafter(np.float32(run), np.float32(0.0)))
+        out[n] = run
+    return out
+
+
+def test_tensor_bound_holds_for_a_truncating_chunk_step_adder():
+    """The "tensor" bound covers the simulated chunk-step adder on random and on
+    cancellation-heavy keys, and is not looser than needed by orders of magnitude."""
+    g = np.random.default_rng(23)
+    mask = (0xFF << 8) | (0x0F << 48)  # one whole and one half chunk
+    chunks = [1, 6]
+    for big in (False, True):
+        qf = g.standard_normal((1, 1, 128)).astype(np.float32)
+        kf = g.standard_normal((1, 120, 1, 128)).astype(np.float32)
+        if big:
+            kf[..., 16:32:2] *= 1e4
+            kf[..., 17:32:2] = -kf[..., 16:32:2] * (qf[0, 0, 16:32:2] / np.where(qf[0, 0, 17:32:2] == 0, 1,
+                                                                                 qf[0, 0, 17:32:2]))
+        q = torch.from_numpy(qf).to(torch.bfloat16)
+        k = torch.from_numpy(kf).to(torch.bfloat16)
+        qd, kd = q.float().numpy()[0, 0].copy(), k.float().numpy()[0, :, 0].copy()
+        dims = [j for i in fasa.pair_list(mask, 128) for j in (2 * i, 2 * i + 1)]
+        keep = np.zeros(128, dtype=bool)
+        keep[dims] = True
+        qd[~keep] = 0.0  # the kernel's B operand is zero outside the dominant pairs
+        exact = fasa.tip_scores(q, k, [120], mask)[0, 0]
+        bound = fasa.score_bound(q, k, [120], mask, model="tensor")[0, 0]
+        got = _chunk_step_sum(qd, kd, chunks)
+        err = np.abs(got - exact)
+        assert np.all(err <= bound), (big, err.max(), bound.min())
+        mag = fasa.score_bound(q, k, [120], mask, model="fma")[0, 0] / (len(dims) * 2.0 ** -24)
+        assert np.all(bound <= 18 * 2.0 ** -23 * 2 * 1.01 * mag + 1e-30)
+
+
 def test_check_selection_accepts_correct_and_rejects_wrong_selections():
     q = _bf16((1, 2, 64), 21)
     k = _bf16((1, 500, 1, 64), 22)
