@@ -266,10 +266,18 @@ atf_status atf_kv_append(const void* k_new, const void* v_new, void* k_cache_chu
  *              below d/2 only.  Only the 8-pair cache chunks holding a dominant
  *              pair are read for the scores.
  *   budget:    keys kept per query head, 1..4096 (all keys when kv_len <= budget).
- * Score of key n for query head h: from +0, every dim j of the dominant pairs
- * in ascending order (2i, then 2i+1) adds its product with one fp32 fused
- * multiply-add, s <- fl(q_j k_j + s); -0 counts as +0.  The kept
- * keys are the `budget` highest scores, equal scores by lower index.  Output:
+ * Score of key n for query head h: the partial dot product of q and k over the
+ * dims of the dominant pairs, summed in fp32 on the tensor cores -- for each
+ * 8-pair cache chunk holding a dominant pair, in ascending order, the chunk's
+ * 16 bf16 products (zero for its non-dominant pairs) are added to the running
+ * sum in one mma.sync step, in a fixed arrangement, so a key's score has the
+ * same bits in every kernel of the call; -0 counts as +0.  (Such a step's
+ * rounding is not documented; the tests hold each score to within
+ * 18 * 2^-23 * (number of dominant chunks) * sum_j |q_j k_j| of the exact one,
+ * and to the exact one where every partial sum is exact, e.g. small integers.)
+ * The kept keys are the `budget` highest scores, equal scores by lower index,
+ * chosen via a threshold from one key in 32 (an exact pass over every key runs
+ * if fewer than `budget` keys reach it).  Output:
  * out[b][h] = softmax over the kept keys of (1/sqrt d) q.k (all d dims), times
  * their values, bf16.
  *   selected:  device int32 [batch][heads][budget] or NULL: the kept key indices,
