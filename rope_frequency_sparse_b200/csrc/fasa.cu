@@ -472,10 +472,10 @@ __global__ void __launch_bounds__(kScoreThreads, 2) fasa_score_kernel(FasaParams
     }
     m &= (hv0 ? 0x55555555u : 0u) | (hv1 ? 0xAAAAAAAAu : 0u);
     if (!__any_sync(0xffffffffu, m != 0u)) continue;
-    // slots: the lanes sharing this lane's two heads (lanes t, t + 4, .., t + 28,
-    // in key order within each tile row) take consecutive runs after the
-    // segment's count; order within a segment is arbitrary (the selection sorts
-    // what it keeps)
+    // slots: the lanes sharing this lane's two heads (lanes t, t + 4, .., t + 28)
+    // take consecutive runs after the segment's count, so each step's candidates
+    // of a head form one block of the list, after the blocks of earlier steps
+    // (the selection orders keys within a block)
     const int c0 = __popc(m & 0x55555555u), c1 = __popc(m & 0xAAAAAAAAu);
     int p0 = c0, p1 = c1;
 #pragma unroll
@@ -580,6 +580,7 @@ struct SegmentList {
 
 struct SelectScratch {
   unsigned int* hist;  // kBins
+  int* warp;           // 32
   int* total;
   int* digit;
   int* gt;
@@ -591,7 +592,7 @@ struct SelectScratch {
 // at or above it in the order of `largest` (descending if true), and writes to
 // *before the number strictly beyond it.  Every thread of the block calls it.
 template <class List, class Val, class In>
-__device__ uint32_t radix_select(const List& list, Val val, In in, int rank, bool largest, int* before,
+__device__ uint32_t radix_select(const List& list, Val val, In in, int rank, bool largest, int* before, int* equal,
                                  const SelectScratch& sc) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t prefix = 0u, pmask = 0u;
@@ -604,12 +605,16 @@ __device__ uint32_t radix_select(const List& list, Val val, In in, int rank, boo
       *sc.gt = 0;
     }
     __syncthreads();
-    for (long long i = tid; i < list.n; i += kSelectThreads) {
-      uint32_t k, x;
-      if (list.get(i, k, x) && in(k, x)) {
+    // one atomic per distinct digit and warp: many entries share their top digits
+    for (long long i0 = 0; i0 < list.n; i0 += kSelectThreads) {
+      const long long i = i0 + tid;
+      uint32_t k, x, d = 0xFFFFFFFFu;
+      if (i < list.n && list.get(i, k, x) && in(k, x)) {
         const uint32_t v = val(k, x);
-        if ((v & pmask) == prefix) atomicAdd(&sc.hist[(v >> shift) & (kBins - 1)], 1u);
+        if ((v & pmask) == prefix) d = (v >> shift) & (kBins - 1);
       }
+      const unsigned int peers = __match_any_sync(0xffffffffu, d);
+      if (d != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&sc.hist[d], static_cast<unsigned int>(__popc(peers)));
     }
     __syncthreads();
     if (warp == 0) {
@@ -643,7 +648,8 @@ __device__ uint32_t radix_select(const List& list, Val val, In in, int rank, boo
     beyond += *sc.gt;
     prefix |= static_cast<uint32_t>(*sc.digit) << shift;
     pmask |= static_cast<uint32_t>(kBins - 1) << shift;
-    __syncthreads();  // digit and gt are rewritten by the next pass
+    if (pass == 3) *equal = static_cast<int>(sc.hist[*sc.digit]);  // entries equal to the whole value
+    __syncthreads();  // digit, gt and the histogram are rewritten by the next pass
   }
   *before = beyond;
   return prefix;
@@ -651,65 +657,217 @@ __device__ uint32_t radix_select(const List& list, Val val, In in, int rank, boo
 
 // Writes to out[0 .. need) the indices of the `need` largest entries of `list`
 // by order key (equal keys: lower index first), ascending, and -1 to out[need ..
-// budget).  The list holds at least `need` entries.
+// budget).  The list holds at least `need` entries, all with indices below L.
+// `bitmap` (bitmap_words words of shared memory, free once the list has been
+// read) orders the kept indices when L fits in it; otherwise they are sorted.
+
 template <class List>
-__device__ void select_emit(const List& list, int need, int budget, int* out, const SelectScratch& sc) {
+__device__ void select_emit(const List& list, int need, int budget, long long L, int* out, uint32_t* bitmap,
+                            int bitmap_words, const SelectScratch& sc) {
   const int tid = threadIdx.x;
   auto by_key = [](uint32_t k, uint32_t) { return k; };
   auto all = [](uint32_t, uint32_t) { return true; };
-  int above = 0;
-  const uint32_t V = radix_select(list, by_key, all, need, true, &above, sc);
+  int above = 0, eq = 0;
+  const uint32_t V = radix_select(list, by_key, all, need, true, &above, &eq, sc);
   const int left = need - above;  // entries equal to V to keep: the lowest indices
-  // count the entries equal to V; if there are more than `left`, the left-th
-  // smallest index among them decides
-  if (tid == 0) *sc.total = 0;
-  __syncthreads();
-  int eq = 0;
-  for (long long i = tid; i < list.n; i += kSelectThreads) {
-    uint32_t k, x;
-    eq += list.get(i, k, x) && k == V;
-  }
-  if (eq) atomicAdd(sc.total, eq);
-  __syncthreads();
   uint32_t I = 0xFFFFFFFFu;
-  if (*sc.total > left) {
+  if (eq > left) {  // the left-th smallest index among the entries equal to V decides
     auto by_idx = [](uint32_t, uint32_t x) { return x; };
     auto equal = [V](uint32_t k, uint32_t) { return k == V; };
-    int below = 0;
-    I = radix_select(list, by_idx, equal, left, false, &below, sc);
+    int below = 0, same = 0;
+    I = radix_select(list, by_idx, equal, left, false, &below, &same, sc);
   }
-  __syncthreads();
+  auto kept = [V, I](uint32_t k, uint32_t x) { return k > V || (k == V && x <= I); };
   if (tid == 0) *sc.total = 0;
   __syncthreads();
-  for (long long i = tid; i < list.n; i += kSelectThreads) {
-    uint32_t k, x;
-    if (list.get(i, k, x) && (k > V || (k == V && x <= I))) {
-      const int slot = atomicAdd(sc.total, 1);
+  const int lane = tid & 31, warp = tid >> 5;
+  for (long long i0 = 0; i0 < list.n; i0 += kSelectThreads) {
+    const long long i = i0 + tid;
+    uint32_t k = 0u, x = 0u;
+    const bool keep = i < list.n && list.get(i, k, x) && kept(k, x);
+    const unsigned int bal = __ballot_sync(0xffffffffu, keep);
+    const int leader = bal ? __ffs(bal) - 1 : 0;
+    int base = 0;
+    if (bal && lane == leader) base = atomicAdd(sc.total, __popc(bal));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (keep) {
+      const int slot = base + __popc(bal & ((1u << lane) - 1u));
       if (slot < need) sc.out[slot] = static_cast<int>(x);
     }
   }
   __syncthreads();
-  // bitonic sort of the kept indices (padded to a power of two)
-  int P = 1;
-  while (P < need) P <<= 1;
-  for (int i = need + tid; i < P; i += kSelectThreads) sc.out[i] = 0x7fffffff;
-  __syncthreads();
-  for (int k = 2; k <= P; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < P; i += kSelectThreads) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const int a = sc.out[i], c = sc.out[ixj];
-          if ((a > c) == ((i & k) == 0)) {
-            sc.out[i] = c;
-            sc.out[ixj] = a;
+  const int nw = static_cast<int>((L + 31) / 32);
+  if (nw <= bitmap_words) {
+    // one bit per key index; warp w then emits the set bits of its run of words,
+    // 32 words at a time (lane l: word 32 j + l of the run), after the counts of
+    // the runs before it
+    for (int i = tid; i < nw; i += kSelectThreads) bitmap[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < need; i += kSelectThreads) {
+      const int x = sc.out[i];
+      if (x >= 0 && x < L) atomicOr(&bitmap[x >> 5], 1u << (x & 31));  // always, with consistent counts
+    }
+    __syncthreads();
+    constexpr int kWarps = kSelectThreads / 32;
+    const int per = (nw + kWarps - 1) / kWarps;
+    const int r0 = min(nw, warp * per), r1 = min(nw, r0 + per);
+    int cnt = 0;
+    for (int w = r0 + lane; w < r1; w += 32) cnt += __popc(bitmap[w]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+    int pos = block_scan(lane == 0 ? cnt : 0, sc.warp, sc.total);
+    pos = __shfl_sync(0xffffffffu, pos, 0);  // this warp's first output slot
+    for (int j = r0; j < r1; j += 32) {
+      const int w = j + lane;
+      const uint32_t bits = w < r1 ? bitmap[w] : 0u;
+      const int c = __popc(bits);
+      int incl = c;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      int q = pos + incl - c;
+      for (uint32_t b = bits; b; b &= b - 1u)
+        if (q < need) out[q++] = 32 * w + __ffs(b) - 1;
+      pos += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  } else {
+    // bitonic sort of the kept indices (padded to a power of two)
+    int P = 1;
+    while (P < need) P <<= 1;
+    for (int i = need + tid; i < P; i += kSelectThreads) sc.out[i] = 0x7fffffff;
+    __syncthreads();
+    for (int k = 2; k <= P; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int i = tid; i < P; i += kSelectThreads) {
+          const int ixj = i ^ j;
+          if (ixj > i) {
+            const int a = sc.out[i], c = sc.out[ixj];
+            if ((a > c) == ((i & k) == 0)) {
+              sc.out[i] = c;
+              sc.out[ixj] = a;
+            }
           }
         }
+        __syncthreads();
       }
-      __syncthreads();
+    }
+    for (int i = tid; i < need; i += kSelectThreads) out[i] = sc.out[i];
+  }
+  for (int i = need + tid; i < budget; i += kSelectThreads) out[i] = -1;
+}
+
+constexpr int kFineBits = 12;                 // bins of the single-pass selection
+constexpr int kFineBins = 1 << kFineBits;
+constexpr int kBoundaryMax = 256;             // keys of the boundary bin ranked exactly
+
+// The shared-memory list as runs, one per thread in thread order (the warp
+// segments: every key of a run is below every key of the next run): keeps the
+// `need` largest keys (equal keys: lower index first) and writes them ascending
+// to out[0 .. need), -1 to out[need .. budget).  One histogram pass of 4096 bins
+// over the 12 bits below the prefix shared by every key (between T and the
+// largest) finds the boundary bin; its keys are ranked exactly against each
+// other, once each, and the kept ones marked in bit 31 of their list index
+// (key indices are below 2^31).  Returns false, having written nothing and
+// marked nothing, if the boundary bin holds more than kBoundaryMax keys.
+// scratch: kFineBins + 3 kBoundaryMax words.
+__device__ bool select_runs(const uint32_t* key, uint32_t* idx, int run_off, int run_len, uint32_t kmin,
+                            uint32_t kmax, int need, int budget, int* out, uint32_t* scratch, const SelectScratch& sc) {
+  const int tid = threadIdx.x;
+  // the bits below the common prefix of kmin and kmax (the whole key if they differ at the top)
+  const uint32_t diff = kmin ^ kmax;
+  const int top = diff ? 32 - __clz(diff) : 1;  // bits that vary: 0 .. top-1
+  const int shift = top > kFineBits ? top - kFineBits : 0;
+  auto bin_of = [kmin, shift](uint32_t k) { return static_cast<int>((k - (kmin >> shift << shift)) >> shift); };
+  // (every key lies in [kmin, kmax]; bin_of is monotone in k and below kFineBins)
+  unsigned int* hist = scratch;
+  uint32_t* bkey = scratch + kFineBins;
+  uint32_t* bidx = bkey + kBoundaryMax;
+  uint32_t* bpos = bidx + kBoundaryMax;
+  for (int i = tid; i < kFineBins; i += kSelectThreads) hist[i] = 0u;
+  __syncthreads();
+  for (int j = 0; j < run_len; ++j) atomicAdd(&hist[bin_of(key[run_off + j])], 1u);
+  __syncthreads();
+  // suffix counts from the top bin: thread t holds bins kFineBins - 4 (t + 1) .. kFineBins - 4 t - 1
+  constexpr int kPer = kFineBins / kSelectThreads;
+  int c[kPer], mine = 0;
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    c[u] = static_cast<int>(hist[kFineBins - kPer * tid - 1 - u]);
+    mine += c[u];
+  }
+  const int before = block_scan(mine, sc.warp, sc.total);  // keys in higher bins than this thread's
+  if (tid == 0) {
+    *sc.digit = -1;
+    *sc.gt = 0;
+  }
+  __syncthreads();
+  if (before < need && need <= before + mine) {
+    int acc = before;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      if (acc + c[u] >= need) {
+        *sc.digit = kFineBins - kPer * tid - 1 - u;  // the boundary bin
+        *sc.gt = acc;                                 // keys above it
+        break;
+      }
+      acc += c[u];
     }
   }
-  for (int i = tid; i < budget; i += kSelectThreads) out[i] = i < need ? sc.out[i] : -1;
+  __syncthreads();
+  const int B = *sc.digit, above = *sc.gt;
+  const int nb = B >= 0 ? static_cast<int>(hist[B]) : 0;
+  if (B < 0 || nb > kBoundaryMax) return false;  // uniform: every thread read the same
+  // the boundary bin's keys, then each one's rank among them (larger key first,
+  // equal keys by lower index): kept if fewer than need - above precede it
+  if (tid == 0) *sc.total = 0;
+  __syncthreads();
+  for (int j = 0; j < run_len; ++j) {
+    const uint32_t k = key[run_off + j];
+    if (bin_of(k) == B) {
+      const int slot = atomicAdd(sc.total, 1);
+      bkey[slot] = k;
+      bidx[slot] = idx[run_off + j];
+      bpos[slot] = static_cast<uint32_t>(run_off + j);
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < nb; e += kSelectThreads) {
+    const uint32_t k = bkey[e], x = bidx[e];
+    int r = 0;
+    for (int f = 0; f < nb; ++f) r += bkey[f] > k || (bkey[f] == k && bidx[f] < x);
+    if (r < need - above) idx[bpos[e]] = x | 0x80000000u;
+  }
+  __syncthreads();
+  auto kept = [&](int j) {
+    const int bn = bin_of(key[run_off + j]);
+    return bn > B || (bn == B && (idx[run_off + j] >> 31));
+  };
+  int nk = 0;
+  for (int j = 0; j < run_len; ++j) nk += kept(j);
+  int pos = block_scan(nk, sc.warp, sc.total);
+  // this run's kept keys in ascending index order after those of the runs before.
+  // A run lists the candidates of each 128-key step of its segment as one block,
+  // steps in ascending order; only within a block are they unordered.
+  for (int j = 0; j < run_len;) {
+    const uint32_t blk = (idx[run_off + j] & 0x7FFFFFFFu) >> 7;
+    int je = j + 1;
+    while (je < run_len && ((idx[run_off + je] & 0x7FFFFFFFu) >> 7) == blk) ++je;
+    int nb_kept = 0;
+    for (int a = j; a < je; ++a) {
+      if (!kept(a)) continue;
+      const uint32_t x = idx[run_off + a] & 0x7FFFFFFFu;
+      int rank = 0;
+      for (int c2 = j; c2 < je; ++c2) rank += kept(c2) && (idx[run_off + c2] & 0x7FFFFFFFu) < x;
+      if (pos + rank < need) out[pos + rank] = static_cast<int>(x);
+      ++nb_kept;
+    }
+    pos += nb_kept;
+    j = je;
+  }
+  for (int i = need + tid; i < budget; i += kSelectThreads) out[i] = -1;
+  return true;
 }
 
 template <int D>
@@ -728,7 +886,9 @@ __global__ void __launch_bounds__(kSelectThreads) fasa_select_kernel(FasaParams 
   __shared__ int s_warp[32];
   __shared__ int s_total, s_digit, s_gt;
   __shared__ int s_out[kMaxFasaBudget];
-  const SelectScratch scr{s_hist, &s_total, &s_digit, &s_gt, s_out};
+  __shared__ uint32_t s_kmax;
+  if (tid == 0) s_kmax = 0u;
+  const SelectScratch scr{s_hist, s_warp, &s_total, &s_digit, &s_gt, s_out};
   const uint32_t T = p.thr[row];
   const long long nseg = (L + kSegKeys - 1) / kSegKeys;
   const unsigned int* cnt = p.seg_cnt + row * p.n_seg;
@@ -745,22 +905,50 @@ __global__ void __launch_bounds__(kSelectThreads) fasa_select_kernel(FasaParams 
     // each group of kSelectThreads segments
     uint32_t* s_key = s_list;
     uint32_t* s_idx = s_list + kSelectCap;
-    int carry = 0;
+    int carry = 0, run_off = 0, run_len = nseg <= kSelectThreads ? 0 : -1;
+    uint32_t kmax = 0u;
     for (long long w0 = 0; w0 < nseg; w0 += kSelectThreads) {
       const long long w = w0 + tid;
       const int cw = w < nseg ? static_cast<int>(cnt[w]) : 0;
       const int off = carry + block_scan(cw, s_warp, &s_total);
-      for (int j = 0; j < cw; ++j) {
-        const uint32_t k = order_key(cscore[w * kSegKeys + j]);
-        s_key[off + j] = k;
-        s_idx[off + j] = cand[w * kSegKeys + j];
-        reached += k >= T;
+      if (run_len >= 0) {  // one segment per thread: its run
+        run_off = off;
+        run_len = cw;
+      }
+      for (int j0 = 0; j0 < cw; j0 += 8) {  // eight entries' loads in flight at a time
+        float sv[8];
+        uint32_t xv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (j0 + u < cw) {
+            sv[u] = cscore[w * kSegKeys + j0 + u];
+            xv[u] = cand[w * kSegKeys + j0 + u];
+          }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (j0 + u < cw) {
+            const uint32_t k = order_key(sv[u]);
+            s_key[off + j0 + u] = k;
+            s_idx[off + j0 + u] = xv[u];
+            reached += k >= T;
+            kmax = max(kmax, k);
+          }
       }
       carry += s_total;
     }
     block_scan(reached, s_warp, &s_total);
     if (s_total >= need) {
-      select_emit(SmemList{s_key, s_idx, m}, need, p.budget, out, scr);
+      // the fast path needs one run per thread, every key at or above T, and room
+      // for its scratch after the key indices (s_idx[m ..])
+      kmax = __reduce_max_sync(0xffffffffu, kmax);
+      if ((tid & 31) == 0) atomicMax(&s_kmax, kmax);
+      __syncthreads();
+      const bool fast = run_len >= 0 && s_total == m && kSelectCap - m >= kFineBins + 3 * kBoundaryMax;
+      if (fast && select_runs(s_key, s_idx, run_off, run_len, T, s_kmax, need, p.budget, out,
+                              s_list + kSelectCap + m, scr))
+        return;
+      // (select_runs wrote nothing; its scratch lay after the list)
+      select_emit(SmemList{s_key, s_idx, m}, need, p.budget, L, out, s_list, 2 * kSelectCap, scr);
       return;
     }
   } else {
@@ -771,7 +959,7 @@ __global__ void __launch_bounds__(kSelectThreads) fasa_select_kernel(FasaParams 
     }
     block_scan(reached, s_warp, &s_total);
     if (s_total >= need) {
-      select_emit(list, need, p.budget, out, scr);
+      select_emit(list, need, p.budget, L, out, s_list, 2 * kSelectCap, scr);
       return;
     }
   }
@@ -802,7 +990,7 @@ __global__ void __launch_bounds__(kSelectThreads) fasa_select_kernel(FasaParams 
     }
   }
   __syncthreads();
-  select_emit(SegmentList{cand, cscore, cnt, L, true}, need, p.budget, out, scr);
+  select_emit(SegmentList{cand, cscore, cnt, L, true}, need, p.budget, L, out, s_list, 2 * kSelectCap, scr);
 }
 
 // 16-byte asynchronous copy global -> shared (completion per thread by
