@@ -44,6 +44,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <mutex>
 #include <cmath>
 #include <cstdint>
 
@@ -91,6 +92,7 @@ struct FasaParams {
   unsigned int* err;        // device error word (bounded waits)
   float* partials;          // [B][Hq][n_split][d + 2]
   int batch, hq, hkv, d, budget, n_split;
+  int b_off;                // first sequence of a launch that covers part of the batch
   long long n_cache, n_seg, seg_cap;  // seg_cap = n_seg * kSegKeys >= n_cache
   unsigned long long mask;  // dominant pairs
   uint32_t chunk_mask;      // bit c: chunk c holds a dominant pair
@@ -351,7 +353,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) fasa_score_kernel(FasaParams
   constexpr int kStepKeys = 16 * NT;
   constexpr uint32_t kStageBytes = kStepKeys * 32;  // one chunk row of each key of a step
   static_assert(kSegKeys % kStepKeys == 0, "a segment is a whole number of steps");
-  const int kvh = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int kvh = blockIdx.y, b = p.b_off + blockIdx.z, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long long L = p.kv_len[b];
   const int need = L < p.budget ? static_cast<int>(L) : p.budget;
   const bool select = need < L;
@@ -872,7 +874,7 @@ __device__ bool select_runs(const uint32_t* key, uint32_t* idx, int run_off, int
 
 template <int D>
 __global__ void __launch_bounds__(kSelectThreads) fasa_select_kernel(FasaParams p) {
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int h = blockIdx.x, b = p.b_off + blockIdx.y, tid = threadIdx.x;
   const long long row = static_cast<long long>(b) * p.hq + h;
   const long long L = p.kv_len[b];
   const int need = L < p.budget ? static_cast<int>(L) : p.budget;
@@ -1013,7 +1015,7 @@ __global__ void __launch_bounds__(kAttendWarps * 32) fasa_attend_kernel(FasaPara
   constexpr int NC = D / 16;
   constexpr int DPL = D / 32;        // dims per lane: 4 (d = 128) or 2 (d = 64)
   constexpr int kGran = D / 8;       // 16-byte pieces of a K row, and of a V row
-  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int split = blockIdx.x, h = blockIdx.y, b = p.b_off + blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.hq / p.hkv, kvh = h / G;
   const long long row = static_cast<long long>(b) * p.hq + h;
@@ -1148,7 +1150,7 @@ __global__ void __launch_bounds__(kAttendWarps * 32) fasa_attend_kernel(FasaPara
 
 template <int D>
 __global__ void __launch_bounds__(D) fasa_combine_kernel(FasaParams p) {
-  const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
+  const int h = blockIdx.x, b = p.b_off + blockIdx.y, e = threadIdx.x;
   const long long row = static_cast<long long>(b) * p.hq + h;
   const float* part = p.partials + row * p.n_split * (D + 2);
   float M = -INFINITY;
@@ -1195,16 +1197,31 @@ FasaLayout fasa_layout(int batch, int heads, long long n_cache, int budget, int 
 }
 
 template <int D, int G>
-void launch_select_path(const FasaParams& p, long long max_len, cudaStream_t s) {
+void launch_front(const FasaParams& p, long long max_len, cudaStream_t s) {
   const size_t hist_smem = static_cast<size_t>(G) * (kHistBins / 2) * sizeof(unsigned int);
   fasa_sample_kernel<D, G><<<dim3(static_cast<unsigned>((max_len + kSampleCtaKeys - 1) / kSampleCtaKeys), p.hkv,
                                   p.batch),
                              kSampleThreads, hist_smem, s>>>(p);
   fasa_threshold_kernel<<<dim3(p.hq, p.batch), kThresholdThreads, 0, s>>>(p);
-  fasa_score_kernel<D, G><<<dim3(static_cast<unsigned>((max_len + kScoreCtaKeys - 1) / kScoreCtaKeys), p.hkv,
-                                 p.batch),
+}
+
+template <int D, int G>
+void launch_score(const FasaParams& p, int nb, long long max_len, cudaStream_t s) {
+  fasa_score_kernel<D, G><<<dim3(static_cast<unsigned>((max_len + kScoreCtaKeys - 1) / kScoreCtaKeys), p.hkv, nb),
                             kScoreThreads, kScoreSmem, s>>>(p);
 }
+
+// Streams and events of the per-sequence chains, per device: created once,
+// used under the mutex (the chains are forked from and joined back to the
+// caller's stream, so two calls must not interleave their records).
+constexpr int kChainStreams = 4;
+struct ChainPool {
+  cudaStream_t st[kChainStreams] = {};
+  cudaEvent_t fork = nullptr, join[kChainStreams] = {};
+  bool ready = false;
+};
+std::mutex g_chain_mu;
+ChainPool g_chain[64];
 
 template <int D>
 cudaError_t launch_fasa(const FasaParams& p, long long max_len, cudaStream_t s) {
@@ -1250,19 +1267,69 @@ cudaError_t launch_fasa(const FasaParams& p, long long max_len, cudaStream_t s) 
     if (e != cudaSuccess) return e;
     if (dev < 64) configured.fetch_or(1ull << dev, std::memory_order_acq_rel);
   }
+  auto score = [&](const FasaParams& q, int nb, long long len, cudaStream_t st) {
+    switch (G) {
+      case 1: launch_score<D, 1>(q, nb, len, st); break;
+      case 2: launch_score<D, 2>(q, nb, len, st); break;
+      case 3: launch_score<D, 3>(q, nb, len, st); break;
+      case 4: launch_score<D, 4>(q, nb, len, st); break;
+      case 5: launch_score<D, 5>(q, nb, len, st); break;
+      case 6: launch_score<D, 6>(q, nb, len, st); break;
+      case 7: launch_score<D, 7>(q, nb, len, st); break;
+      default: launch_score<D, 8>(q, nb, len, st); break;
+    }
+  };
+  // select -> attention -> combine for sequences b_off .. b_off + nb - 1
+  auto finish = [&](const FasaParams& q, int nb, cudaStream_t st) {
+    fasa_select_kernel<D><<<dim3(q.hq, nb), kSelectThreads, kSelectSmem, st>>>(q);
+    fasa_attend_kernel<D><<<dim3(q.n_split, q.hq, nb), kAttendWarps * 32, kAttendSmem, st>>>(q);
+    fasa_combine_kernel<D><<<dim3(q.hq, nb), D, 0, st>>>(q);
+  };
   switch (G) {
-    case 1: launch_select_path<D, 1>(p, max_len, s); break;
-    case 2: launch_select_path<D, 2>(p, max_len, s); break;
-    case 3: launch_select_path<D, 3>(p, max_len, s); break;
-    case 4: launch_select_path<D, 4>(p, max_len, s); break;
-    case 5: launch_select_path<D, 5>(p, max_len, s); break;
-    case 6: launch_select_path<D, 6>(p, max_len, s); break;
-    case 7: launch_select_path<D, 7>(p, max_len, s); break;
-    default: launch_select_path<D, 8>(p, max_len, s); break;
+    case 1: launch_front<D, 1>(p, max_len, s); break;
+    case 2: launch_front<D, 2>(p, max_len, s); break;
+    case 3: launch_front<D, 3>(p, max_len, s); break;
+    case 4: launch_front<D, 4>(p, max_len, s); break;
+    case 5: launch_front<D, 5>(p, max_len, s); break;
+    case 6: launch_front<D, 6>(p, max_len, s); break;
+    case 7: launch_front<D, 7>(p, max_len, s); break;
+    default: launch_front<D, 8>(p, max_len, s); break;
   }
-  fasa_select_kernel<D><<<dim3(p.hq, p.batch), kSelectThreads, kSelectSmem, s>>>(p);
-  fasa_attend_kernel<D><<<dim3(p.n_split, p.hq, p.batch), kAttendWarps * 32, kAttendSmem, s>>>(p);
-  fasa_combine_kernel<D><<<dim3(p.hq, p.batch), D, 0, s>>>(p);
+  if (p.batch == 1 || dev >= 64) {
+    score(p, p.batch, max_len, s);
+    finish(p, p.batch, s);
+    return cudaGetLastError();
+  }
+  // one chain (score -> select -> attention -> combine) per sequence on the
+  // library's streams: the chains' latency-bound selections and attention
+  // overlap other chains' bandwidth-bound scoring
+  std::lock_guard<std::mutex> lk(g_chain_mu);
+  ChainPool& pool = g_chain[dev];
+  if (!pool.ready) {
+    for (int i = 0; i < kChainStreams && e == cudaSuccess; ++i) {
+      e = cudaStreamCreateWithFlags(&pool.st[i], cudaStreamNonBlocking);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&pool.join[i], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&pool.fork, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+    pool.ready = true;
+  }
+  e = cudaEventRecord(pool.fork, s);
+  const int used = p.batch < kChainStreams ? p.batch : kChainStreams;
+  for (int i = 0; i < used && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(pool.st[i], pool.fork, 0);
+  if (e != cudaSuccess) return e;
+  for (int b = 0; b < p.batch; ++b) {
+    FasaParams q = p;
+    q.b_off = b;
+    cudaStream_t st = pool.st[b % kChainStreams];
+    score(q, 1, p.kv_len[b], st);
+    finish(q, 1, st);
+  }
+  for (int i = 0; i < used && e == cudaSuccess; ++i) {
+    e = cudaEventRecord(pool.join[i], pool.st[i]);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, pool.join[i], 0);
+  }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
