@@ -89,6 +89,8 @@ struct FasaParams {
   unsigned int* hist;       // [B][Hq][kHistBins] sample histograms
   uint32_t* thr;            // [B][Hq] threshold T as an order-preserving key
   int* sel;                 // [B][Hq][budget], ascending, -1 padded
+  float* sel_score;         // [B][Hq][budget]: the kept keys' TIP scores (rows with sel_has_score)
+  int* sel_has_score;       // [B][Hq]: 1 if the row's sel_score is written
   unsigned int* err;        // device error word (bounded waits)
   float* partials;          // [B][Hq][n_split][d + 2]
   int batch, hq, hkv, d, budget, n_split;
@@ -775,7 +777,8 @@ constexpr int kBoundaryMax = 256;             // keys of the boundary bin ranked
 // marked nothing, if the boundary bin holds more than kBoundaryMax keys.
 // scratch: kFineBins + 3 kBoundaryMax words.
 __device__ bool select_runs(const uint32_t* key, uint32_t* idx, int run_off, int run_len, uint32_t kmin,
-                            uint32_t kmax, int need, int budget, int* out, uint32_t* scratch, const SelectScratch& sc) {
+                            uint32_t kmax, int need, int budget, int* out, float* out_score, uint32_t* scratch,
+                            const SelectScratch& sc) {
   const int tid = threadIdx.x;
   // the bits below the common prefix of kmin and kmax (the whole key if they differ at the top)
   const uint32_t diff = kmin ^ kmax;
@@ -862,7 +865,10 @@ __device__ bool select_runs(const uint32_t* key, uint32_t* idx, int run_off, int
       const uint32_t x = idx[run_off + a] & 0x7FFFFFFFu;
       int rank = 0;
       for (int c2 = j; c2 < je; ++c2) rank += kept(c2) && (idx[run_off + c2] & 0x7FFFFFFFu) < x;
-      if (pos + rank < need) out[pos + rank] = static_cast<int>(x);
+      if (pos + rank < need) {
+        out[pos + rank] = static_cast<int>(x);
+        out_score[pos + rank] = key_float(key[run_off + a]);
+      }
       ++nb_kept;
     }
     pos += nb_kept;
@@ -879,6 +885,7 @@ __global__ void __launch_bounds__(kSelectThreads) fasa_select_kernel(FasaParams 
   const long long L = p.kv_len[b];
   const int need = L < p.budget ? static_cast<int>(L) : p.budget;
   int* out = p.sel + row * p.budget;
+  if (tid == 0) p.sel_has_score[row] = 0;  // set to 1 by the path that writes the scores
   if (need == L) {  // every key is selected, already in order
     for (int i = tid; i < p.budget; i += kSelectThreads) out[i] = i < L ? i : -1;
     return;
@@ -947,8 +954,10 @@ __global__ void __launch_bounds__(kSelectThreads) fasa_select_kernel(FasaParams 
       __syncthreads();
       const bool fast = run_len >= 0 && s_total == m && kSelectCap - m >= kFineBins + 3 * kBoundaryMax;
       if (fast && select_runs(s_key, s_idx, run_off, run_len, T, s_kmax, need, p.budget, out,
-                              s_list + kSelectCap + m, scr))
+                              p.sel_score + row * p.budget, s_list + kSelectCap + m, scr)) {
+        if (tid == 0) p.sel_has_score[row] = 1;
         return;
+      }
       // (select_runs wrote nothing; its scratch lay after the list)
       select_emit(SmemList{s_key, s_idx, m}, need, p.budget, L, out, s_list, 2 * kSelectCap, scr);
       return;
@@ -1029,6 +1038,15 @@ __global__ void __launch_bounds__(kAttendWarps * 32) fasa_attend_kernel(FasaPara
   __nv_bfloat16* sv = sk + 32 * D;
   const int n_mine = lane < nk ? p.sel[row * p.budget + j0 + lane] : -1;
   const bool ok = n_mine >= 0 && n_mine < L;  // always, with consistent inputs
+  // With the kept keys' TIP scores at hand (the partial dot products over the
+  // dominant pairs), only the other pairs are summed here: the chunks whose
+  // eight pairs are all dominant are not read at all.
+  const bool tip = p.sel_has_score[row] != 0;
+  const float s_tip = tip && lane < nk ? p.sel_score[row * p.budget + j0 + lane] : 0.f;
+  uint32_t full_chunks = 0u;  // bit c: chunk c entirely dominant (skipped when tip)
+  if (tip)
+#pragma unroll
+    for (int c = 0; c < NC; ++c) full_chunks |= static_cast<uint32_t>(((p.mask >> (8 * c)) & 0xFFu) == 0xFFu) << c;
   const __nv_bfloat16* kb = p.kc + (static_cast<long long>(b) * p.hkv + kvh) * NC * p.n_cache * 16;
   const __nv_bfloat16* vb = p.v + static_cast<long long>(b) * p.n_cache * p.hkv * D + kvh * D;
   // piece i of the warp's copy: key i / (2 kGran), then its K pieces, then its V pieces
@@ -1038,6 +1056,7 @@ __global__ void __launch_bounds__(kAttendWarps * 32) fasa_attend_kernel(FasaPara
     const bool kok = __shfl_sync(0xffffffffu, static_cast<int>(ok), key) != 0;
     if (!kok) continue;
     if (gi < kGran) {  // K: chunk gi / 2, half gi % 2
+      if ((full_chunks >> (gi >> 1)) & 1u) continue;
       const __nv_bfloat16* src = kb + (static_cast<long long>(gi >> 1) * p.n_cache + n) * 16 + 8 * (gi & 1);
       cp_async16(sk + key * D + 8 * gi, src);
     } else {
@@ -1052,13 +1071,17 @@ __global__ void __launch_bounds__(kAttendWarps * 32) fasa_attend_kernel(FasaPara
   const float scale = kLog2e * rsqrtf(static_cast<float>(D));
   float q[DPL];
 #pragma unroll
-  for (int e = 0; e < DPL; ++e) q[e] = __bfloat162float(p.q[row * D + DPL * lane + e]) * scale;
+  for (int e = 0; e < DPL; ++e) {
+    q[e] = __bfloat162float(p.q[row * D + DPL * lane + e]) * scale;
+    if (tip && ((p.mask >> ((DPL * lane + e) / 2)) & 1ull)) q[e] = 0.f;  // in the TIP score already
+  }
+  const bool lane_reads = !((full_chunks >> ((DPL * lane) / 16)) & 1u);  // this lane's K dims were copied
   // partial dot products of all 32 keys over this lane's dims
   float dp[32];
 #pragma unroll
   for (int k = 0; k < 32; ++k) {
     float acc = 0.f;
-    if (k < nk) {
+    if (k < nk && lane_reads) {
       const __nv_bfloat16* kr = sk + k * D + DPL * lane;
       if constexpr (DPL == 4) {
         const uint2 w = *reinterpret_cast<const uint2*>(kr);
@@ -1088,7 +1111,7 @@ __global__ void __launch_bounds__(kAttendWarps * 32) fasa_attend_kernel(FasaPara
     }
   }
   const bool live = lane < nk && ok;
-  const float sdot = live ? dp[0] : -INFINITY;
+  const float sdot = live ? fmaf(s_tip, scale, dp[0]) : -INFINITY;
   float mrun = sdot;
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) mrun = fmaxf(mrun, __shfl_xor_sync(0xffffffffu, mrun, off));
@@ -1169,7 +1192,7 @@ __global__ void __launch_bounds__(D) fasa_combine_kernel(FasaParams p) {
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct FasaLayout {
-  size_t cand, cand_score, seg_cnt, hist, thr, sel, partials, total;
+  size_t cand, cand_score, seg_cnt, hist, thr, sel, sel_score, sel_has_score, partials, total;
 };
 
 FasaLayout fasa_layout(int batch, int heads, long long n_cache, int budget, int d, bool own_sel) {
@@ -1190,6 +1213,10 @@ FasaLayout fasa_layout(int batch, int heads, long long n_cache, int budget, int 
   off += align256(rows * sizeof(uint32_t));
   L.sel = off;
   off += own_sel ? 0 : align256(rows * budget * sizeof(int));
+  L.sel_score = off;
+  off += align256(rows * budget * sizeof(float));
+  L.sel_has_score = off;
+  off += align256(rows * sizeof(int));
   L.partials = off;
   off += align256(rows * n_split * (d + 2) * sizeof(float));
   L.total = off;
@@ -1393,6 +1420,8 @@ extern "C" atf_status atf_fasa_decode(const void* q_rot, const void* k_chunked, 
   p.err = device_error_word();
   if (!p.err) return report_error(ATF_ERR_CUDA, "fasa: no CUDA device / device error word unavailable");
   p.partials = reinterpret_cast<float*>(ws + Lw.partials);
+  p.sel_score = reinterpret_cast<float*>(ws + Lw.sel_score);
+  p.sel_has_score = reinterpret_cast<int*>(ws + Lw.sel_has_score);
   p.batch = batch;
   p.hq = heads;
   p.hkv = kv_heads;

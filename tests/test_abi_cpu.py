@@ -175,13 +175,14 @@ def test_workspace_sizes(lib):
     assert atf.atf_prefill_host_workspace_bytes(0, 1000, 1500, 28, 4, 128, 0) == 0
     # FASA: candidate indices and scores per (sequence, query head, key slot of the 1024-key warp segments),
     # a count per segment, 4096-bin sample histograms, the thresholds (padded to 256 bytes), the selected
-    # indices, attention partials (128 selected keys per split)
+    # indices and their scores, a flag per row, attention partials (128 selected keys per split)
     fws = atf.atf_fasa_workspace_bytes(4, 28, 1 << 20, 2048, 128)
     rows = 4 * 28
-    assert fws == (rows * (1 << 20) * 8 + rows * 1024 * 4 + rows * 4096 * 4 + 512 + rows * 2048 * 4
+    assert fws == (rows * (1 << 20) * 8 + rows * 1024 * 4 + rows * 4096 * 4 + 512 + 2 * rows * 2048 * 4 + 512
                    + rows * 16 * 130 * 4)
     # a cache that is not a whole number of segments rounds up to one
-    assert atf.atf_fasa_workspace_bytes(1, 1, 1000, 10, 64) == 1024 * 8 + 256 + 4096 * 4 + 256 + 256 + 512
+    assert atf.atf_fasa_workspace_bytes(1, 1, 1000, 10, 64) == (1024 * 8 + 256 + 4096 * 4 + 256 + 256 + 256 + 256
+                                                                 + 512)
     dws = atf.atf_decode_workspace_bytes(4, 28, 4, 1 << 20, 128)
     assert dws % (4 * 28 * 130 * 4) == 0 and dws > 0
 
