@@ -22,31 +22,35 @@
 //      all keys score at or above T.
 //   3. fasa_score_kernel: one CTA per (8192 keys, kv head, sequence); each warp
 //      owns a segment of 1024 consecutive keys, 128 at a time (8 tiles of 16
-//      keys x all query heads of the kv head).  It reads only the 8-pair chunks
-//      that hold a dominant pair (32 bytes per key and chunk, one 8-byte load
-//      per lane and tile row) and appends the keys scoring at or above T, with
-//      their scores, to the segment's list of that head.
+//      keys x all query heads of the kv head), the keys' chunk rows brought in
+//      by a per-warp ring of bulk copies.  It reads only the 8-pair chunks that
+//      hold a dominant pair and appends the keys scoring at or above T, with
+//      their scores, to the segment's list of that head, each 128-key step's
+//      candidates as one block after the earlier steps'.
 //   4. fasa_select_kernel: one CTA per (query head, sequence) gathers the
-//      segments' lists into shared memory, finds the budget-th largest score by a
-//      radix select on the scores' order-preserving bits (and, among keys equal
-//      to it, the lowest indices by a second one on the index), and sorts the
-//      kept indices.  If fewer than `budget` keys reached T (the sample was not
-//      representative), it recomputes every key's score the same way and
-//      selects over all of them; a list longer than shared memory is selected in
-//      place.
+//      segments' lists into shared memory; one 4096-bin histogram pass finds the
+//      bin holding the budget-th largest score, whose keys are ranked exactly
+//      (larger score, then lower index); every thread then writes its segment's
+//      kept keys in index order, with their TIP scores.  A crowded boundary bin
+//      or a list longer than shared memory takes radix passes instead; if fewer
+//      than `budget` keys reached T (the sample was not representative), every
+//      key's score is recomputed the same way and the selection runs over all.
 //   5. fasa_attend_kernel: (split of 128 selected keys, query head, sequence);
 //      each warp copies its 32 keys' K rows (chunk-major pieces) and V rows into
 //      shared memory with asynchronous copies, all in flight at once, computes
 //      their 32 dot products together and a softmax over them; partials as in
-//      the split decode.
+//      the split decode.  With the TIP scores, chunks whose pairs are all
+//      dominant are not read (the TIP score is their part of q.k).
 //   6. fasa_combine_kernel: merges the splits (log-sum-exp) into bf16 output.
+// Kernels 1 and 2 run once over the batch; 3 to 6 run as one chain per sequence
+// on library streams forked from and joined back to the caller's stream.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
-#include <mutex>
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/atf.h"
 #include "atf_internal.cuh"
