@@ -159,6 +159,46 @@ def test_fasa_without_optional_outputs_gives_the_same_result():
     assert torch.equal(out1, out2)
 
 
+def test_fasa_more_sequences_than_chain_streams():
+    """Each sequence's scoring, selection and attention run as one chain on the
+    library's streams, round robin over four: six sequences of mixed lengths reuse
+    two of them."""
+    q, k, v = _inputs(6, 2600, 8, 2, 128, seed=73)
+    _check(q, k, v, [2600, 1, 1300, 2600, 700, 2599], LOW16, 300)
+
+
+def test_fasa_captured_in_a_graph_matches_direct_calls():
+    """The call forks its chains from the caller's stream and joins them back, so
+    it captures into a CUDA graph; replays give the direct call's output and
+    selection bit for bit."""
+    B, N, Hq, Hkv, d, budget = 5, 3000, 28, 4, 128, 256
+    q, k, v = _inputs(B, N, Hq, Hkv, d, seed=79)
+    kv_len = [3000, 2999, 1000, 2048, 77]
+    qd, kd, vd = q.cuda(), _chunked(k), v.cuda()
+    wsb = atf.atf_fasa_workspace_bytes(B, Hq, N, budget, d)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(qd)
+    sel = torch.empty((B, Hq, budget), dtype=torch.int32, device="cuda")
+
+    def call():
+        atf.atf_fasa_decode(qd, kd, vd, out, B, kv_len, N, Hq, Hkv, d, LOW16, budget, sel, None, ws, wsb, None)
+
+    call()
+    torch.cuda.synchronize()
+    atf.atf_check()
+    out_ref, sel_ref = out.clone(), sel.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    for _ in range(2):
+        out.zero_()
+        sel.fill_(-3)
+        graph.replay()
+        torch.cuda.synchronize()
+        atf.atf_check()
+        assert torch.equal(out, out_ref) and torch.equal(sel, sel_ref)
+
+
 def test_fasa_full_size_cache():
     """One sequence of the 4 x 2^20-token decode workload, 28 query heads, budget 2048."""
     N, budget = 1 << 20, 2048
