@@ -286,6 +286,11 @@ atf_status atf_kv_append(const void* k_new, const void* v_new, void* k_cache_chu
  *              n >= kv_len[b] are not written).
  *   workspace: device scratch of atf_fasa_workspace_bytes(...) bytes (the
  *              size assumes selected is NULL; less is needed when it is given).
+ * Streams: with batch > 1 the work of each sequence runs on one of four
+ * streams the library creates on the device's first such call (kept for the
+ * process, so they do not survive cudaDeviceReset), forked from `stream` and
+ * joined back to it with events: the call stays ordered on `stream` and can be
+ * captured into a CUDA graph.
  * Errors: d not 64/128, more than 8 query heads per kv head, batch above 64,
  * budget outside [1, 4096] -> ATF_ERR_UNSUPPORTED; bad sizes, mask or kv_len,
  * small workspace, null or misaligned pointers -> ATF_ERR_INVALID_ARG. */
