@@ -328,15 +328,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(sQ + g * C::TILE_BYTES + bx * (BN * 128), &tm_q, &sh->q_full[g], bx * 64, h, t0 + g * BM, b);
       }
       int k_issued = 0, v_issued = 0;
+      // Only the active chunk columns of K are loaded: the first 64-dim box (pairs
+      // 0-31) is skipped for a tile where pair 31's window, the widest of them, is
+      // below every query-key distance of every Q tile that reads the tile (Q tile g
+      // at KV tile j spans centre(j + g) +- (BN - 1)).  Then no MMA issues those
+      // chunks (its depth starts past every pair with W_i < centre - 48) and no
+      // boundary correction reads them (none of them straddles).
+      const long long w_box0 = SPARSE && C::BOXES > 1 ? static_cast<long long>(sh->w[31]) : 0x7fffffffffffffffLL;
       for (int j = 0; j < T; ++j) {
         const int n0 = static_cast<int>(tile_n0(j));
         {
           const int s = j % NSK, use = j / NSK;
           if (j >= NSK && !mbar_wait(&sh->k_empty[s], (use - 1) & 1, abort, p.err, 0x101)) break;
-          mbar_arrive_expect_tx(&sh->k_full[s], C::TILE_BYTES);
+          long long dmin = 0x7fffffffffffffffLL;
+          for (int g = 0; g < nq; ++g)
+            if (j >= jstart(g)) dmin = min(dmin, centre(j + g) - (BN - 1));
+          const int bx0 = w_box0 < dmin ? 1 : 0;
+          mbar_arrive_expect_tx(&sh->k_full[s], C::TILE_BYTES / C::BOXES * (C::BOXES - bx0));
 #pragma unroll
           for (int bx = 0; bx < C::BOXES; ++bx)
-            tma_load_4d(sK + s * C::TILE_BYTES + bx * (BN * 128), &tm_k, &sh->k_full[s], bx * 64, hk, n0, b);
+            if (bx >= bx0)
+              tma_load_4d(sK + s * C::TILE_BYTES + bx * (BN * 128), &tm_k, &sh->k_full[s], bx * 64, hk, n0, b);
           k_issued = j + 1;
         }
         {
