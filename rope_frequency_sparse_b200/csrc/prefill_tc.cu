@@ -125,6 +125,15 @@ constexpr int smem_bytes() {
 // keeps both kinds of correction small, and must be <= 1 so that the pairs added
 // back on a tile were zeroed at the step just before it (a(j+1) >= z(j)).
 constexpr int kZeroOffset = -48;
+// A warp's clean tile (every pair dead for all of its elements or live for all of
+// them, nothing zeroed after it) holds no window W_i >= lo within [lo, lo + kCleanSpan),
+// lo = center + 32q - 127 its smallest distance: the span covers the tile's own
+// distances (lo .. lo + BN + 30) and reaches the next tile's zero point
+// (lo + 2 BN - 1 + kZeroOffset), so no pair dies during a run of clean tiles and
+// the zeroed pairs after the run are still those before it.
+constexpr int kCleanSpan = 2 * BN - 1 + kZeroOffset;
+static_assert(kZeroOffset <= 1 && kCleanSpan >= BN + 31,
+              "zero point between the tile's element distances and the next tile's add-back range");
 
 // The window table held across a warp: lane l keeps W_l and W_{l+32} (a pair
 // index past the head's pairs holds a sentinel that is never below a threshold).
@@ -775,12 +784,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
 
       // Tiles are visited from the diagonal towards key 0.  A run of clean tiles
-      // for this warp ends at the first tile whose distance range [lo, lo + 207)
+      // for this warp ends at the first tile whose range [lo, lo + kCleanSpan)
       // -- lo = centre + 32 quarter - 127, the smallest distance of the warp's
-      // elements; lo + 207 reaches the next tile's zero point -- holds some window
-      // W_i: there a boundary crosses the warp's elements or pairs die next tile.
-      // The first window not below lo is the next one to enter that range (W is
-      // non-decreasing), so the run length follows from it directly.
+      // elements -- holds some window W_i: there a boundary crosses the warp's
+      // elements or pairs die next tile.  The first window not below lo is the
+      // next one to enter that range (W is non-decreasing), so the run length
+      // follows from it directly.
       int j = j0;
       while (ok && j < T) {
         int jn = T, a_run = 0;
@@ -790,7 +799,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (a_run >= C::NP) {
             jn = j;  // every pair dead: the correcting body handles tiles without S
           } else {
-            const long long excess = ww.at(a_run) - lo - 206;  // tile j + t holds W when 128 t >= excess
+            const long long excess = ww.at(a_run) - lo - (kCleanSpan - 1);  // tile j + t holds W when BN t >= excess
             jn = excess <= 0 ? j : j + static_cast<int>(min((excess + BN - 1) / BN, static_cast<long long>(T - j)));
           }
         }
